@@ -1,0 +1,188 @@
+/*
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged-KV decode library.
+ *
+ * Two operations of one decode step of a vLLM-style serving engine:
+ *
+ *  1. paged_kv_cache_write ("reshape_and_cache"): scatter this step's new K/V
+ *     vectors into their physical slots of the paged KV cache.
+ *  2. paged_gqa_decode_attention: grouped-query attention of one new query
+ *     token per sequence over that sequence's cached keys and values, read
+ *     through a PagedAttention block table, with an optional split-KV
+ *     (flash-decoding) mode whose partial softmaxes are merged by the
+ *     log-sum-exp rule inside the same launch.
+ *
+ * Sources, cited by page title and section:
+ *  - "rvLLM 소개" (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3:
+ *    the KV cache is managed by PagedAttention through block tables; attention
+ *    is grouped-query, Qwen2.5's 12 query heads sharing 2 KV heads, and
+ *    serving every query head of a KV head from one read of that head's K/V
+ *    is what cuts KV bandwidth 6x; the cache is f16, FP8 E4M3 optionally.
+ *  - same page, §CUDA 그래프 리플레이: decode steps are replayed from CUDA
+ *    graphs on the caller's stream, after the per-step upload of block tables
+ *    and context lengths. Hence every call here takes a stream, reads no
+ *    device data on the host, allocates nothing and never synchronises, so
+ *    it can be captured into a graph.
+ *  - vLLM talk summary (aitrends.kr), §용어 해설 (KV Cache, PagedAttention):
+ *    the cache keeps the keys and values of earlier tokens in fixed-size
+ *    pages mapped like OS virtual memory.
+ * The pages state no layout, argument list or numerical convention; the
+ * ones below are this library's readings, listed with each function.
+ *
+ * Common conventions
+ *  - All pointers are DEVICE pointers (cudaMalloc'd or equivalent) unless a
+ *    comment says otherwise. The caller owns every buffer, the workspace
+ *    included. The library allocates no device memory.
+ *  - Layouts are dense row-major (C order), innermost dimension last:
+ *      q, out        [B, Hq, D]                   float16
+ *      k/v cache     [num_blocks, block_size, Hkv, D]  float16, or uint8 E4M3
+ *      k/v new       [T, Hkv, D]                  float16
+ *      block_tables  [B, max_blocks_per_seq]      int32 (physical block ids)
+ *      context_lens  [B]                          int32
+ *      slot_mapping  [T]                          int64
+ *    Query head h reads KV head h / (Hq / Hkv) (contiguous groups).
+ *    Token t of sequence b lives in physical block block_tables[b][t / bs],
+ *    row t % bs. context_lens[b] counts every token attended to, this step's
+ *    token included. Rows past context_lens[b] and table entries past
+ *    ceil(context_lens[b] / bs) are never read and may hold anything.
+ *  - FP8 caches use OCP E4M3 ("FN": bias 7, max 448, no infinities) with one
+ *    fp32 scale per tensor: stored = RNE_satfinite(x / scale) (division in
+ *    fp32), value = decoded * scale.
+ *  - v1 supports D == 128, block_size == 16, 1 <= Hq/Hkv <= 8, and pointers
+ *    aligned to 16 bytes; other shapes return PKV_ERR_UNSUPPORTED.
+ *  - Argument errors are detected on the host, before any launch, and
+ *    returned synchronously. A failed launch returns PKV_ERR_CUDA (the CUDA
+ *    error is left set, readable with cudaGetLastError). Device data (table
+ *    entries, lengths, slots) is not read on the host; kernels clamp or skip
+ *    values outside the pool and record them in a device error word that
+ *    pkv_device_error() returns.
+ *  - Every call is asynchronous with respect to the host and ordered on
+ *    `stream` (a cudaStream_t; NULL = legacy default stream).
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+    PKV_ERR_UNSUPPORTED = 2,   /* valid but not implemented in this version */
+    PKV_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    PKV_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
+} pkv_status;
+
+typedef enum {
+    PKV_KV_F16 = 0,            /* float16 cache */
+    PKV_KV_FP8_E4M3 = 1        /* uint8 OCP E4M3 cache with per-tensor scales */
+} pkv_kv_dtype;
+
+/* Bits of the device error word (pkv_device_error). */
+#define PKV_DEVERR_CONTEXT_LEN   0x1u  /* a context length exceeded max_context_len or the
+                                          table capacity; it was clamped */
+#define PKV_DEVERR_BLOCK_ID      0x2u  /* a table entry lay outside [0, num_blocks); its
+                                          block read as zeros */
+#define PKV_DEVERR_SLOT          0x4u  /* a slot lay outside the pool; the token was skipped */
+#define PKV_DEVERR_WAIT_TIMEOUT  0x8u  /* an on-chip barrier wait ran out of its time limit */
+
+/*
+ * paged_kv_cache_write -- reshape_and_cache.
+ *
+ * For each token i < num_tokens with s = slot_mapping[i] >= 0, writes
+ *   k_cache[s / block_size][s % block_size][h][:] = k_new[i][h][:]   for all h < Hkv
+ * and the same for V. An FP8 cache stores E4M3 codes of k_new / k_scale
+ * (v_new / v_scale), rounded to nearest even and saturated to +-448; the
+ * scales are ignored for an f16 cache. Negative slots are skipped (padding).
+ * Slots at or beyond num_blocks * block_size are skipped and flagged
+ * (PKV_DEVERR_SLOT). Two tokens with the same slot: the result is one of
+ * them, unspecified which. f16 writes are bit-exact copies.
+ *
+ * Arguments: k_new, v_new [T, Hkv, D] f16; k_cache, v_cache as above;
+ * slot_mapping [T] int64; scales > 0 and finite when kv_dtype is FP8.
+ * num_tokens == 0 is a no-op returning PKV_OK.
+ */
+pkv_status paged_kv_cache_write(const void* k_new, const void* v_new,
+                                void* k_cache, void* v_cache,
+                                const int64_t* slot_mapping,
+                                int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t num_blocks, int32_t block_size,
+                                int32_t kv_dtype, float k_scale, float v_scale,
+                                void* stream);
+
+/*
+ * Bytes of workspace paged_gqa_decode_attention needs for these sizes:
+ * 0 when partition_tokens == 0 (single pass), else partial results of
+ * ceil(max_context_len / partition_tokens) partitions per (sequence, query
+ * head) plus one counter per (sequence, KV head). Returns 0 for invalid sizes.
+ */
+size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads,
+                                       int32_t num_kv_heads, int32_t head_dim,
+                                       int32_t max_context_len, int32_t partition_tokens);
+
+/*
+ * A partition size for split-KV that gives the GPU enough independent work:
+ * a multiple of block_size chosen from the batch, KV heads, the longest
+ * context and the SM count (sm_count <= 0: query the current device).
+ * Returns 0 (single pass) when splitting would not add parallelism.
+ */
+int32_t paged_gqa_decode_suggest_partition(int32_t batch, int32_t num_kv_heads,
+                                           int32_t max_context_len, int32_t block_size,
+                                           int32_t sm_count);
+
+/*
+ * paged_gqa_decode_attention -- one decode step of grouped-query attention.
+ *
+ * For every sequence b < batch and query head h < Hq, with g = h / (Hq/Hkv)
+ * and L = context_lens[b]:
+ *   s_t    = softmax_scale * dot(q[b][h], K_t)                     t < L
+ *   out[b][h] = sum_t softmax(s)_t * V_t                           (f16, RNE)
+ * where K_t = k_cache[block_tables[b][t / bs]][t % bs][g] (times k_scale for
+ * FP8) and likewise V_t. L == 0 gives an all-zero row. Accumulation is fp32.
+ *
+ * partition_tokens == 0: one pass per (sequence, KV head).
+ * partition_tokens  > 0: a multiple of block_size; tokens [p*P, (p+1)*P) form
+ *   partition p, each partition computes its own (max, sum, output) and the
+ *   last partition of a (sequence, KV head) to finish merges them:
+ *   M = max m_p, w_p = l_p * exp(m_p - M), out = sum w_p o_p / sum w_p.
+ *   `workspace` must then hold paged_gqa_decode_workspace_size(...) bytes,
+ *   256-byte aligned, and must be ZERO-FILLED before its first use; every
+ *   call leaves it ready for the next one (its counters back at zero), so a
+ *   workspace is allocated and cleared once and reused. Calls that share a
+ *   workspace must not run concurrently on different streams.
+ *
+ * max_context_len must be >= every context_lens[b] (larger lengths are
+ * clamped and flagged) and <= max_blocks_per_seq * block_size.
+ * num_blocks is the pool size; table entries outside it read zeros and are
+ * flagged. The value of softmax_scale is used as given (e.g. 1/sqrt(D)).
+ */
+pkv_status paged_gqa_decode_attention(void* out, const void* q,
+                                      const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t block_size,
+                                      int32_t max_blocks_per_seq, int32_t num_blocks,
+                                      int32_t max_context_len, float softmax_scale,
+                                      int32_t kv_dtype, float k_scale, float v_scale,
+                                      int32_t partition_tokens,
+                                      void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/* Static text for a status code. Never NULL. */
+const char* pkv_status_string(pkv_status status);
+
+/*
+ * Reads and clears the device error word of the current device (PKV_DEVERR_*
+ * bits) into *flags. Synchronous: waits for all prior work on the device.
+ * Must not be called while a stream is being captured.
+ */
+pkv_status pkv_device_error(uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

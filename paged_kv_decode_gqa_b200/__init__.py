@@ -1,0 +1,170 @@
+"""Paged GQA decode attention and paged KV-cache write for B200 (sm_100a).
+
+A thin ctypes binding over the C ABI declared in ``include/pagedkv.h`` and
+implemented by the in-tree CUDA library ``libpagedkv_b200.so``. The functions
+here only marshal arguments (shapes, device pointers, the current CUDA stream)
+and raise on a non-OK status: every step of the computation runs in the
+library's kernels. There is no CPU fallback; importing this package fails if
+the library has not been built (``python -m paged_kv_decode_gqa_b200.build``).
+
+Tensors are torch CUDA tensors used as plain device memory:
+  q, out            [B, Hq, D]              float16
+  k_cache, v_cache  [NB, block_size, Hkv, D] float16, or uint8 (FP8 E4M3 codes)
+  k_new, v_new      [T, Hkv, D]             float16
+  block_tables      [B, max_blocks]         int32
+  context_lens      [B]                     int32
+  slot_mapping      [T]                     int64
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libpagedkv_b200.so")
+
+_P, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+_SIGNATURES = {
+    "paged_kv_cache_write": ([_P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32, _P],
+                             ctypes.c_int),
+    "paged_gqa_decode_workspace_size": ([_i32, _i32, _i32, _i32, _i32, _i32], _sz),
+    "paged_gqa_decode_suggest_partition": ([_i32, _i32, _i32, _i32, _i32], _i32),
+    "paged_gqa_decode_attention": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                    _i32, _f32, _i32, _f32, _f32, _i32, _P, _sz, _P], ctypes.c_int),
+    "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "pkv_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+}
+# The symbols include/pagedkv.h declares (checked by the CPU tests).
+EXPORTED = tuple(_SIGNATURES)
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """The CUDA library, loaded on first use. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY_PATH):
+            raise ImportError(
+                f"CUDA library not built: {LIBRARY_PATH} is missing "
+                "(run `python -m paged_kv_decode_gqa_b200.build`)")
+        lib = ctypes.CDLL(LIBRARY_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return load_library()
+    raise AttributeError(name)
+
+
+PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_WORKSPACE, PKV_ERR_CUDA = range(5)
+PKV_KV_F16, PKV_KV_FP8_E4M3 = 0, 1
+DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+_KV_DTYPES = {"f16": PKV_KV_F16, "fp8": PKV_KV_FP8_E4M3}
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        text = load_library().pkv_status_string(status).decode()
+        super().__init__(f"{where}: {text} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != PKV_OK:
+        raise PagedKVError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _dense(name, t, *dtypes):
+    """Checks that `t` is a dense CUDA tensor of one of `dtypes` (names)."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if str(t.dtype).replace("torch.", "") not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(dtypes)}, got {t.dtype}")
+
+
+def kv_dtype_code(kv_dtype: str) -> int:
+    try:
+        return _KV_DTYPES[kv_dtype]
+    except KeyError:
+        raise ValueError(f"kv_dtype must be one of {sorted(_KV_DTYPES)}") from None
+
+
+def paged_kv_cache_write(k_new, v_new, k_cache, v_cache, slot_mapping, *, kv_dtype="f16",
+                         k_scale=1.0, v_scale=1.0, stream=None) -> None:
+    """reshape_and_cache: k_cache[slot // bs, slot % bs] = k_new[i] (and V)."""
+    cdt = "uint8" if kv_dtype == "fp8" else "float16"
+    for n, t in (("k_new", k_new), ("v_new", v_new)):
+        _dense(n, t, "float16")
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _dense(n, t, cdt)
+    _dense("slot_mapping", slot_mapping, "int64")
+    T, Hkv, D = k_new.shape
+    NB, bs = k_cache.shape[0], k_cache.shape[1]
+    _check(load_library().paged_kv_cache_write(
+        _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, NB,
+        bs, kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _stream(stream)),
+        "paged_kv_cache_write")
+
+
+def paged_gqa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                    partition_tokens) -> int:
+    return int(load_library().paged_gqa_decode_workspace_size(
+        batch, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens))
+
+
+def paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len, block_size=16,
+                                       sm_count=0) -> int:
+    return int(load_library().paged_gqa_decode_suggest_partition(
+        batch, num_kv_heads, max_context_len, block_size, sm_count))
+
+
+def paged_gqa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, *,
+                               max_context_len, softmax_scale, kv_dtype="f16", k_scale=1.0,
+                               v_scale=1.0, partition_tokens=0, workspace=None, stream=None) -> None:
+    """out[b, h] = softmax(scale * q[b, h] . K^T) V over the paged context of b."""
+    cdt = "uint8" if kv_dtype == "fp8" else "float16"
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    _dense("k_cache", k_cache, cdt)
+    _dense("v_cache", v_cache, cdt)
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    if workspace is not None:
+        _dense("workspace", workspace, "uint8", "float32", "int32")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load_library().paged_gqa_decode_attention(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(softmax_scale),
+        kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), int(partition_tokens),
+        _ptr(workspace), ws_bytes, _stream(stream)), "paged_gqa_decode_attention")
+
+
+def pkv_device_error() -> int:
+    """Reads and clears the device error word (DEVERR_* bits). Synchronises the device."""
+    flags = ctypes.c_uint32(0)
+    _check(load_library().pkv_device_error(ctypes.byref(flags)), "pkv_device_error")
+    return int(flags.value)

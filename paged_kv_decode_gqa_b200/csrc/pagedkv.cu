@@ -1,0 +1,300 @@
+// C ABI of the paged-KV decode library (declared in include/pagedkv.h):
+// argument checks, TMA descriptors, launch planning and launches. The whole
+// library is this one translation unit, so the device error word needs no
+// relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "pagedkv.h"
+#include "cache_write.cuh"
+#include "decode_attention.cuh"
+
+namespace {
+
+using pkv::kHeadDim;
+using pkv::kPageRows;
+
+constexpr int kConsumers = 4;
+constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
+constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// View of one cache tensor [num_blocks, 16, Hkv, 128] as a 3-D TMA tensor
+// (channel, head, pool row) with 16-row x 128-byte boxes, 128-byte swizzled.
+bool make_cache_map(CUtensorMap* map, const void* base, bool fp8, int num_blocks, int Hkv) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+    if (!encode) return false;
+    const cuuint64_t esz = fp8 ? 1 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hkv, (cuuint64_t)num_blocks * kPageRows};
+    cuuint64_t strides[2] = {kHeadDim * esz, (cuuint64_t)Hkv * kHeadDim * esz};
+    cuuint32_t box[3] = {fp8 ? 128u : 64u, 1u, (cuuint32_t)kPageRows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Small per-thread cache of encoded maps: serving loops reuse the same pool.
+struct MapKey {
+    const void* base;
+    int num_blocks, Hkv;
+    bool fp8;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && num_blocks == o.num_blocks && Hkv == o.Hkv && fp8 == o.fp8;
+    }
+};
+
+bool cached_cache_map(CUtensorMap* out, const void* base, bool fp8, int num_blocks, int Hkv) {
+    constexpr int kSlots = 8;
+    thread_local MapKey keys[kSlots];
+    thread_local CUtensorMap maps[kSlots];
+    thread_local int used = 0, next = 0;
+    const MapKey key{base, num_blocks, Hkv, fp8};
+    for (int i = 0; i < used; ++i)
+        if (keys[i] == key) {
+            *out = maps[i];
+            return true;
+        }
+    CUtensorMap m;
+    if (!make_cache_map(&m, base, fp8, num_blocks, Hkv)) return false;
+    keys[next] = key;
+    maps[next] = m;
+    next = (next + 1) % kSlots;
+    used = std::min(used + 1, kSlots);
+    *out = m;
+    return true;
+}
+
+// Opt a kernel into its dynamic shared memory once per device.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, unsigned long long* done_mask) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_ACQ_REL);
+    return e;
+}
+
+template <bool kFp8, int kStages>
+pkv_status launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
+                         int B, int Hkv, cudaStream_t stream) {
+    using S = pkv::DecodeShape<kFp8, kConsumers, kStages>;
+    auto kernel = pkv::decode_attention_kernel<kFp8, kConsumers, kStages>;
+    static unsigned long long done = 0;
+    if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
+    dim3 grid(prm.nparts, Hkv, B);
+    kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(mk, mv, prm);
+    return cudaPeekAtLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+struct WorkspaceLayout {
+    size_t o, m, l, count, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t nparts) {
+    WorkspaceLayout w{};
+    const int64_t rows = B * Hq * nparts;
+    w.o = 0;
+    w.m = w.o + align256(rows * kHeadDim * sizeof(float));
+    w.l = w.m + align256(rows * sizeof(float));
+    w.count = w.l + align256(rows * sizeof(float));
+    w.total = w.count + align256(B * Hkv * sizeof(unsigned int));
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status status) {
+    switch (status) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case PKV_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+pkv_status pkv_device_error(uint32_t* flags) {
+    if (!flags) return PKV_ERR_INVALID_ARG;
+    unsigned int v = 0, zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, pkv::g_device_error, sizeof(v)) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemcpyToSymbol(pkv::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return PKV_ERR_CUDA;
+    *flags = v;
+    return PKV_OK;
+}
+
+pkv_status paged_kv_cache_write(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                                const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t num_blocks, int32_t block_size,
+                                int32_t kv_dtype, float k_scale, float v_scale, void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (head_dim % 8 != 0) return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+        return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    pkv::CacheWriteParams prm;
+    prm.k_new = static_cast<const uint4*>(k_new);
+    prm.v_new = static_cast<const uint4*>(v_new);
+    prm.k_cache = k_cache;
+    prm.v_cache = v_cache;
+    prm.slot_mapping = slot_mapping;
+    prm.num_slots = (int64_t)num_blocks * block_size;
+    prm.num_tokens = num_tokens;
+    prm.chunks_per_token = num_kv_heads * (head_dim / 8);
+    prm.k_scale = k_scale;
+    prm.v_scale = v_scale;
+    const int64_t total = (int64_t)num_tokens * prm.chunks_per_token;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fp8)
+        pkv::cache_write_kernel<true><<<(unsigned)blocks, threads, 0, st>>>(prm);
+    else
+        pkv::cache_write_kernel<false><<<(unsigned)blocks, threads, 0, st>>>(prm);
+    return cudaPeekAtLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t max_context_len,
+                                       int32_t partition_tokens) {
+    if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim ||
+        max_context_len < 0 || partition_tokens < 0)
+        return 0;
+    if (partition_tokens == 0) return 0;
+    const int64_t nparts = std::max<int64_t>(1, (max_context_len + partition_tokens - 1) / partition_tokens);
+    return workspace_layout(batch, num_q_heads, num_kv_heads, nparts).total;
+}
+
+int32_t paged_gqa_decode_suggest_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
+                                           int32_t block_size, int32_t sm_count) {
+    if (batch <= 0 || num_kv_heads <= 0 || max_context_len <= 0 || block_size <= 0) return 0;
+    if (sm_count <= 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            sm_count = 148;
+    }
+    // Aim for about eight partitions per resident CTA slot (two per SM),
+    // assuming contexts spread up to max_context_len (mean about half of it).
+    const double work = (double)batch * num_kv_heads * (0.5 * max_context_len);
+    const double want = 16.0 * sm_count;
+    int32_t P = 128;
+    while (P < 4096 && work / (2.0 * P) >= want) P *= 2;
+    P = std::max(P, block_size);
+    P -= P % block_size;
+    if (P >= max_context_len) return 0;
+    return P;
+}
+
+pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                                      int32_t num_blocks, int32_t max_context_len, float softmax_scale,
+                                      int32_t kv_dtype, float k_scale, float v_scale,
+                                      int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_tokens < 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return PKV_ERR_INVALID_ARG;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != kHeadDim || block_size != kPageRows) return PKV_ERR_UNSUPPORTED;
+    const int G = num_q_heads / num_kv_heads;
+    if (G > pkv::kGroupPad) return PKV_ERR_UNSUPPORTED;
+    if (partition_tokens % block_size != 0) return PKV_ERR_INVALID_ARG;
+    if (batch == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PKV_ERR_INVALID_ARG;
+    if (batch > 65535 || num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
+
+    // plan: a partition covering the longest context is a single pass
+    int32_t P = partition_tokens;
+    if (P == 0 || P >= max_context_len) P = std::max(max_context_len, 1);
+    P = (P + kPageRows - 1) / kPageRows * kPageRows;
+    const int nparts = std::max(1, (max_context_len + P - 1) / P);
+
+    pkv::DecodeParams prm{};
+    prm.out = static_cast<__half*>(out);
+    prm.q = static_cast<const __half*>(q);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    if (nparts > 1) {
+        const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, num_kv_heads, nparts);
+        if (!workspace || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        prm.ws_o = reinterpret_cast<float*>(ws + wl.o);
+        prm.ws_m = reinterpret_cast<float*>(ws + wl.m);
+        prm.ws_l = reinterpret_cast<float*>(ws + wl.l);
+        prm.ws_count = reinterpret_cast<unsigned int*>(ws + wl.count);
+    }
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.G = G;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition_tokens = P;
+    prm.nparts = nparts;
+    const float log2e = 1.4426950408889634f;
+    prm.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
+    prm.out_scale = fp8 ? v_scale : 1.f;
+
+    CUtensorMap mk, mv;
+    if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
+        !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
+        return PKV_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return fp8 ? launch_decode<true, kStagesFp8>(prm, mk, mv, batch, num_kv_heads, st)
+               : launch_decode<false, kStagesF16>(prm, mk, mv, batch, num_kv_heads, st);
+}
+
+}  // extern "C"

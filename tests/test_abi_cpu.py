@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every entry point include/pagedkv.h declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_decode_gqa_b200 as pkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_entry_points():
+    assert declared_functions() == sorted(pkv.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = pkv.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    lib = pkv.load_library()
+    for code in range(5):
+        assert lib.pkv_status_string(code)
+    assert lib.pkv_status_string(99) == b"unknown status"
+
+
+def test_workspace_size():
+    assert pkv.paged_gqa_decode_workspace_size(8, 28, 4, 128, 32768, 0) == 0
+    n = pkv.paged_gqa_decode_workspace_size(8, 28, 4, 128, 32768, 512)
+    rows = 8 * 28 * 64
+    assert n >= rows * 128 * 4 + 2 * rows * 4 + 8 * 4
+    assert n % 256 == 0
+    assert pkv.paged_gqa_decode_workspace_size(8, 28, 4, 64, 32768, 512) == 0   # D != 128
+
+
+def test_suggest_partition_is_a_multiple_of_the_page():
+    for B, Hkv, L in [(64, 2, 2048), (128, 4, 4096), (256, 2, 8192), (8, 4, 32768), (1, 1, 64)]:
+        P = pkv.paged_gqa_decode_suggest_partition(B, Hkv, L, 16, 148)
+        assert P == 0 or (P % 16 == 0 and 16 <= P < L)
+    assert pkv.paged_gqa_decode_suggest_partition(2, 2, 40, 16, 148) == 0
+
+
+# Fake but aligned device pointers: every call below must be rejected by the
+# host-side checks, before the library touches CUDA.
+A = 1 << 20
+
+
+def _attn(**kw):
+    args = dict(out=A, q=A, k=A, v=A, bt=A, cl=A, B=2, Hq=12, Hkv=2, D=128, bs=16, mb=4, NB=64,
+                maxlen=40, scale=0.088, dt=0, ks=1.0, vs=1.0, P=0, ws=0, wsb=0)
+    args.update(kw)
+    a = args
+    return pkv.load_library().paged_gqa_decode_attention(
+        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"],
+        a["mb"], a["NB"], a["maxlen"], a["scale"], a["dt"], a["ks"], a["vs"], a["P"], a["ws"], a["wsb"],
+        None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(out=A + 8), pkv.PKV_ERR_INVALID_ARG),            # misaligned
+    (dict(Hq=13), pkv.PKV_ERR_INVALID_ARG),                # Hq % Hkv != 0
+    (dict(Hq=20), pkv.PKV_ERR_UNSUPPORTED),                # group of 10 > 8
+    (dict(D=64), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(bs=32, mb=2), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(maxlen=65), pkv.PKV_ERR_INVALID_ARG),            # > max_blocks * bs
+    (dict(P=20), pkv.PKV_ERR_INVALID_ARG),                 # not a multiple of bs
+    (dict(P=16), pkv.PKV_ERR_WORKSPACE),                   # split without workspace
+    (dict(P=16, ws=A, wsb=64), pkv.PKV_ERR_WORKSPACE),     # too small
+    (dict(dt=1, ks=0.0), pkv.PKV_ERR_INVALID_ARG),         # FP8 needs positive scales
+    (dict(dt=7), pkv.PKV_ERR_INVALID_ARG),
+    (dict(B=-1), pkv.PKV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), pkv.PKV_ERR_INVALID_ARG),
+    (dict(B=0), pkv.PKV_OK),                                # empty batch: nothing to do
+])
+def test_attention_rejects_bad_arguments_on_host(kw, status):
+    assert _attn(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k_new=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(D=12), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(dt=1, ks=-1.0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(slots=A + 4), pkv.PKV_ERR_INVALID_ARG),
+    (dict(T=0), pkv.PKV_OK),
+])
+def test_cache_write_rejects_bad_arguments_on_host(kw, status):
+    a = dict(k_new=A, v_new=A, kc=A, vc=A, slots=A, T=4, Hkv=2, D=128, NB=64, bs=16, dt=0,
+             ks=1.0, vs=1.0)
+    a.update(kw)
+    rc = pkv.load_library().paged_kv_cache_write(a["k_new"], a["v_new"], a["kc"], a["vc"], a["slots"],
+                                                 a["T"], a["Hkv"], a["D"], a["NB"], a["bs"], a["dt"],
+                                                 a["ks"], a["vs"], None)
+    assert rc == status
+
+
+def test_pages_head_counts_give_the_6x_kv_read_cut():
+    """The GQA read saving the page quotes is Hq/Hkv under the byte model bench.py reports."""
+    import json
+    import bench
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "qwen25_gqa_heads.json")))
+    lens = [100, 2048, 17]
+    grouped = bench.kv_bytes(lens, g["Hkv"], 128, 2)
+    per_query_head = bench.kv_bytes(lens, g["Hq"], 128, 2)
+    assert per_query_head / grouped == g["kv_bandwidth_reduction"]

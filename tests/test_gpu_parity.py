@@ -1,0 +1,310 @@
+"""Parity of the CUDA path (through the C-ABI binding) with the float64 oracle.
+
+Cache write: bit-exact. Attention: max |gpu - oracle| <= 2e-3 and <= 1e-2 of
+max |oracle| (FP8: the oracle runs on the same E4M3 bytes). Sizes span several
+stages of the shared-memory ring and ragged last blocks; the full workload
+sizes run in the launch configuration the benchmark times, checked on sampled
+sequences.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_gqa_b200 as pkv
+import workloads as W
+from _gpu_helpers import DecodeRun, assert_attention_close, dev, fp8_caches, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clear_device_error():
+    pkv.pkv_device_error()
+    yield
+    torch.cuda.synchronize()
+
+
+def _run(w, seed, kv_dtype=None):
+    x = W.make_inputs(w, seed)
+    kv_dtype = kv_dtype or w.kv_dtype
+    if kv_dtype == "fp8":
+        kq, vq = fp8_caches(x)
+        return DecodeRun(w, x, "fp8", kq, vq)
+    return DecodeRun(w, x)
+
+
+# ------------------------------------------------------------------ cache write
+def _cache_write_case(w, seed, kv_dtype):
+    x = W.make_inputs(w, seed)
+    if kv_dtype == "fp8":
+        kc, vc = fp8_caches(x)
+    else:
+        kc, vc = x["k_pool"], x["v_pool"]
+    slots = x["slot_mapping"].copy()
+    if slots.size > 2:
+        slots[1] = -1                                       # padding token: skipped
+    k_dev, v_dev = dev(kc), dev(vc)
+    pkv.paged_kv_cache_write(dev(x["k_new"]), dev(x["v_new"]), k_dev, v_dev, dev(slots),
+                             kv_dtype=kv_dtype, k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    kr, vr = kc.copy(), vc.copy()
+    oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, slots, kv_dtype=kv_dtype,
+                                k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    view = (lambda a: a.view(np.uint16)) if kv_dtype == "f16" else (lambda a: a)
+    assert np.array_equal(view(host(k_dev)), view(kr))
+    assert np.array_equal(view(host(v_dev)), view(vr))
+    assert pkv.pkv_device_error() == 0
+
+
+@pytest.mark.parametrize("kv_dtype", ["f16", "fp8"])
+def test_cache_write_tiny_bit_exact(kv_dtype):
+    _cache_write_case(W.WORKLOADS["tiny"], 0, kv_dtype)
+
+
+@pytest.mark.parametrize("kv_dtype", ["f16", "fp8"])
+def test_cache_write_7b_step_bit_exact(kv_dtype):
+    """128 new tokens into the full 32k-block pool (Qwen2.5-7B shape), whole caches compared."""
+    w = W.WORKLOADS["qwen2.5-7b"]
+    if kv_dtype == "fp8":
+        w = W.with_sizes(w, kv_dtype="fp8")
+    _cache_write_case(w, 1, kv_dtype)
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.0078125, 0.0133, 3.7])
+def test_cache_write_fp8_every_f16_value(scale):
+    """Every finite f16 value (and +-inf, NaN) through the device quantiser, compared bytewise."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16)
+    n = -(-vals.size // 128) * 128
+    flat = np.zeros(n, dtype=np.float16)
+    flat[:vals.size] = vals
+    T = n // 128
+    k_new = flat.reshape(T, 1, 128)
+    v_new = k_new[::-1].copy()
+    NB = -(-T // 16)
+    kc = np.zeros((NB, 16, 1, 128), np.uint8)
+    vc = np.zeros_like(kc)
+    slots = np.arange(T, dtype=np.int64)
+    k_dev, v_dev = dev(kc), dev(vc)
+    pkv.paged_kv_cache_write(dev(k_new), dev(v_new), k_dev, v_dev, dev(slots), kv_dtype="fp8",
+                             k_scale=scale, v_scale=scale)
+    kr, vr = kc.copy(), vc.copy()
+    oracle.paged_kv_cache_write(k_new, v_new, kr, vr, slots, kv_dtype="fp8", k_scale=scale,
+                                v_scale=scale)
+    assert np.array_equal(host(k_dev), kr)
+    assert np.array_equal(host(v_dev), vr)
+
+
+def test_cache_write_flags_slot_outside_pool():
+    kc = torch.zeros((4, 16, 1, 128), dtype=torch.float16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kn = torch.ones((2, 1, 128), dtype=torch.float16, device="cuda")
+    slots = torch.tensor([3, 64], dtype=torch.int64, device="cuda")
+    pkv.paged_kv_cache_write(kn, kn, kc, vc, slots)
+    assert pkv.pkv_device_error() == pkv.DEVERR_SLOT
+    assert kc[0, 3].eq(1).all() and kc.sum().item() == 128
+
+
+# ------------------------------------------------------------- attention parity
+@pytest.mark.parametrize("P", [0, 16, 32])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_config_f16(P, seed):
+    r = _run(W.WORKLOADS["tiny"], seed)
+    assert_attention_close(host(r.attention(P)), r.oracle(), f"tiny P={P}")
+    assert pkv.pkv_device_error() == 0
+
+
+REDUCED = {
+    "qwen2.5-1.5b": dict(B=8),
+    "qwen2.5-7b": dict(B=6, num_blocks=2048),
+    "fp8-e4m3": dict(B=4, num_blocks=4096, ctx=("uniform", 17, 2600)),
+    "skewed-split": dict(B=4, num_blocks=1024, ctx=("skewed", 4100, 3, 1, 700)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(REDUCED))
+@pytest.mark.parametrize("P", [0, 64, 512])
+def test_reduced_configs(name, P):
+    w = W.with_sizes(W.WORKLOADS[name], **REDUCED[name])
+    for seed in (0, 3):
+        r = _run(w, seed)
+        assert_attention_close(host(r.attention(P)), r.oracle(), f"{name} P={P} seed={seed}")
+    assert pkv.pkv_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["qwen2.5-1.5b", "qwen2.5-7b", "fp8-e4m3", "skewed-split"])
+def test_full_size_configs_sampled(name):
+    """Full workload on the device in the benchmark's plan; oracle on sampled sequences."""
+    w = W.WORKLOADS[name]
+    r = _run(w, 0)
+    lens = r.x["context_lens"]
+    rng = np.random.default_rng(5)
+    seqs = sorted(set([int(np.argmax(lens)), int(np.argmin(lens))]
+                      + list(rng.choice(w.B, size=min(w.B, 6), replace=False))))
+    ref = r.oracle(seqs=seqs)
+    P_bench = w.partition_tokens or pkv.paged_gqa_decode_suggest_partition(w.B, w.Hkv, r.max_len)
+    for P in sorted({0, P_bench}):
+        out = host(r.attention(P))
+        assert_attention_close(out[seqs], ref, f"{name} P={P}")
+    assert pkv.pkv_device_error() == 0
+
+
+# ------------------------------------------------------- invariants and edges
+def test_context_one_is_exactly_v0():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=5, num_blocks=64, ctx=("fixed", (1, 1, 1, 1, 1)))
+    r = _run(w, 2)
+    out = host(r.attention())
+    for b in range(w.B):
+        blk = r.x["block_tables"][b, 0]
+        v0 = r.x["v_pool"][blk, 0]                          # [Hkv, D]
+        assert np.array_equal(out[b].view(np.uint16), np.repeat(v0, w.group, axis=0).view(np.uint16))
+
+
+def test_block_permutation_invariance_bitwise():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=6, num_blocks=1024)
+    r = _run(w, 4)
+    out1 = host(r.attention(128))
+    perm = np.random.default_rng(9).permutation(w.num_blocks)
+    k2 = np.empty_like(r.k_host); v2 = np.empty_like(r.v_host)
+    k2[perm] = r.k_host; v2[perm] = r.v_host
+    bt = r.x["block_tables"]
+    bt2 = np.where(bt >= 0, perm[np.maximum(bt, 0)], -1).astype(np.int32)
+    out2 = host(r.attention(128, bt=dev(bt2), k=dev(k2), v=dev(v2)))
+    assert np.array_equal(out1.view(np.uint16), out2.view(np.uint16))
+
+
+def test_split_with_partition_covering_context_is_bitwise_single_pass():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=4, num_blocks=2048)
+    r = _run(w, 6)
+    single = host(r.attention(0))
+    P = -(-r.max_len // 16) * 16
+    assert np.array_equal(single.view(np.uint16), host(r.attention(P)).view(np.uint16))
+
+
+def test_split_equals_single_within_tolerance_and_workspace_reuse():
+    w = W.with_sizes(W.WORKLOADS["skewed-split"], B=4, num_blocks=1024, ctx=("skewed", 5000, 3, 16, 900))
+    r = _run(w, 7)
+    ref = r.oracle()
+    B, Hq, D = r.q.shape
+    n = pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, 256)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):                                      # the same workspace, reused
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device="cuda")
+        pkv.paged_gqa_decode_attention(out, r.q, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                                       softmax_scale=float(r.x["softmax_scale"]), partition_tokens=256,
+                                       workspace=ws)
+        outs.append(host(out))
+    for o in outs:
+        assert_attention_close(o, ref, "split 256")
+        assert np.array_equal(o.view(np.uint16), outs[0].view(np.uint16))
+    assert_attention_close(host(r.attention(0)), ref, "single")
+
+
+def test_poison_never_read_bitwise():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=6, num_blocks=2048, ctx=("uniform", 1, 300))
+    xa = W.make_inputs(w, 8, poison=True)
+    xb = W.make_inputs(w, 8, poison=False)
+    ra, rb = DecodeRun(w, xa), DecodeRun(w, xb)
+    for P in (0, 64):
+        a, b = host(ra.attention(P)), host(rb.attention(P))
+        assert np.isfinite(a.astype(np.float32)).all()
+        assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_fp8_poison_code_never_read():
+    w = W.with_sizes(W.WORKLOADS["fp8-e4m3"], B=5, num_blocks=1024, ctx=("uniform", 1, 200))
+    x = W.make_inputs(w, 9)
+    kq, vq = fp8_caches(x)                                  # NaN rows quantise to 0x7F
+    assert (kq == 0x7F).any()
+    r = DecodeRun(w, x, "fp8", kq, vq)
+    for P in (0, 32):
+        assert_attention_close(host(r.attention(P)), r.oracle(), f"fp8 poison P={P}")
+
+
+def test_head_map_contiguous_groups():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=3, num_blocks=1024)
+    x = W.make_inputs(w, 10, poison=False)
+    x["v_pool"][:] = np.arange(w.Hkv, dtype=np.float16)[None, None, :, None]
+    r = DecodeRun(w, x)
+    out = host(r.attention(64)).astype(np.float64)
+    expect = np.repeat(np.arange(w.Hkv, dtype=np.float64), w.group)[None, :, None]
+    assert np.array_equal(out, np.broadcast_to(expect, out.shape))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (16, 4), (14, 2), (8, 1), (32, 4)])
+def test_group_sizes(Hq, Hkv):
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=3, Hq=Hq, Hkv=Hkv, num_blocks=1024,
+                     ctx=("uniform", 1, 1000))
+    r = _run(w, 11)
+    for P in (0, 128):
+        assert_attention_close(host(r.attention(P)), r.oracle(), f"Hq={Hq} Hkv={Hkv} P={P}")
+
+
+def test_empty_contexts_give_zero_rows():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=4, num_blocks=512, ctx=("fixed", (0, 33, 0, 700)))
+    r = _run(w, 12)
+    for P in (0, 64):
+        out = host(r.attention(P))
+        assert not out[0].any() and not out[2].any()
+        assert_attention_close(out, r.oracle(), f"empty P={P}")
+
+
+def test_all_contexts_empty_and_zero_max_len():
+    w = W.with_sizes(W.WORKLOADS["tiny"], ctx=("fixed", (0, 0)))
+    r = _run(w, 0)
+    out = host(r.attention(0, max_len=0))
+    assert not out.any()
+
+
+def test_bad_block_id_and_length_are_flagged_not_faulted():
+    w = W.with_sizes(W.WORKLOADS["tiny"])
+    r = _run(w, 1)
+    bt = r.x["block_tables"].copy()
+    bt[1, 0] = w.num_blocks + 5                              # outside the pool: reads zeros
+    r.attention(0, bt=dev(bt))
+    assert pkv.pkv_device_error() == pkv.DEVERR_BLOCK_ID
+    cl = r.x["context_lens"].copy()
+    cl[0] = 10_000                                           # beyond max_context_len: clamped
+    r.attention(0, cl=dev(cl))
+    # clamped to 40 tokens, sequence 0 (17 live tokens) also reaches its unused
+    # third table entry (-1), which is flagged as well
+    assert pkv.pkv_device_error() == pkv.DEVERR_CONTEXT_LEN | pkv.DEVERR_BLOCK_ID
+
+
+def test_step_captured_in_cuda_graph():
+    """Cache write + attention captured once and replayed on the caller's stream."""
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=8, num_blocks=2048)
+    x = W.make_inputs(w, 13)
+    r = DecodeRun(w, x)
+    P = 128
+    B, Hq, D = r.q.shape
+    ws = torch.zeros(pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, P),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, Hq, D), dtype=torch.float16, device="cuda")
+    kn, vn, sl = dev(x["k_new"]), dev(x["v_new"]), dev(x["slot_mapping"])
+
+    def step():
+        pkv.paged_kv_cache_write(kn, vn, r.k, r.v, sl)
+        pkv.paged_gqa_decode_attention(out, r.q, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                                       softmax_scale=float(x["softmax_scale"]), partition_tokens=P,
+                                       workspace=ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()                                               # warm-up (attribute set-up, maps)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    kr, vr = x["k_pool"].copy(), x["v_pool"].copy()
+    oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"])
+    ref = oracle.paged_gqa_decode(x["q"], kr, vr, x["block_tables"], x["context_lens"],
+                                  float(x["softmax_scale"]))
+    assert_attention_close(host(out), ref, "graph replay")
+    del g
