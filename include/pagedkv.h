@@ -181,6 +181,47 @@ const char* pkv_status_string(pkv_status status);
  */
 pkv_status pkv_device_error(uint32_t* flags);
 
+/*
+ * Size of the library-owned split-KV scratch used by
+ * paged_gqa_decode_attention_static_workspace (8 MiB per GPU).
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (8u << 20)
+
+/*
+ * paged_gqa_decode_attention_static_workspace -- the same attention as
+ * paged_gqa_decode_attention, for callers that cannot allocate device memory.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * such as a serving engine that hands (nearly) all free GPU memory to its KV
+ * cache pool at start-up (the `--gpu-memory-utilization 0.90` setting the
+ * rvLLM page shows) and owns no allocator for per-call scratch, a step being
+ * recorded into a CUDA graph where cudaMalloc must not be called, or a
+ * foreign-language caller with no access to the process's allocator.
+ *
+ * Arguments are those of paged_gqa_decode_attention without the workspace.
+ * The split-KV scratch is a fixed PKV_STATIC_WORKSPACE_BYTES array inside the
+ * library (a file-scope __device__ array: every GPU that loads the library
+ * holds it until the process exits). Nothing is allocated and no allocating
+ * library routine is called.
+ *  - Sizes whose split-KV scratch, paged_gqa_decode_workspace_size(...),
+ *    exceeds PKV_STATIC_WORKSPACE_BYTES are rejected with PKV_ERR_WORKSPACE
+ *    before any launch; single-pass calls need no scratch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents; each call clears the part that must start at zero (its
+ *    partition counters) on `stream` before launching. Calls whose execution
+ *    overlaps on the GPU (other streams, other threads) race on the array and
+ *    give undefined results: serialise them.
+ */
+pkv_status paged_gqa_decode_attention_static_workspace(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+    int32_t max_context_len, float softmax_scale, int32_t kv_dtype,
+    float k_scale, float v_scale, int32_t partition_tokens, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,6 +33,9 @@ _SIGNATURES = {
                                     _i32, _f32, _i32, _f32, _f32, _i32, _P, _sz, _P], ctypes.c_int),
     "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "pkv_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "paged_gqa_decode_attention_static_workspace": (
+        [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _f32,
+         _f32, _i32, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -168,3 +171,35 @@ def pkv_device_error() -> int:
     flags = ctypes.c_uint32(0)
     _check(load_library().pkv_device_error(ctypes.byref(flags)), "pkv_device_error")
     return int(flags.value)
+
+
+# Size of the library's own split-KV scratch (PKV_STATIC_WORKSPACE_BYTES).
+STATIC_WORKSPACE_BYTES = 8 << 20
+
+
+def paged_gqa_decode_attention_static_workspace(out, q, k_cache, v_cache, block_tables,
+                                                context_lens, *, max_context_len, softmax_scale,
+                                                kv_dtype="f16", k_scale=1.0, v_scale=1.0,
+                                                partition_tokens=0, stream=None) -> None:
+    """paged_gqa_decode_attention without a caller workspace, for callers that
+    cannot allocate device memory (an engine that gave all free HBM to its KV
+    pool, a step being captured into a CUDA graph, a foreign-language caller
+    without the process's allocator). Split-KV scratch comes from a fixed
+    STATIC_WORKSPACE_BYTES array inside the library, shared by every call on a
+    device: calls must not overlap on the GPU. Sizes needing more scratch raise
+    PagedKVError (workspace). The first call on a device looks up the array's
+    address and should come before any stream capture."""
+    cdt = "uint8" if kv_dtype == "fp8" else "float16"
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    _dense("k_cache", k_cache, cdt)
+    _dense("v_cache", v_cache, cdt)
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    _check(load_library().paged_gqa_decode_attention_static_workspace(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(softmax_scale),
+        kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), int(partition_tokens),
+        _stream(stream)), "paged_gqa_decode_attention_static_workspace")

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -298,3 +299,66 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Split-KV scratch owned by the library, for callers that cannot allocate.
+// The host name of this array is only a stand-in for it: kernels get its
+// device address, looked up once per device below.
+static __device__ __align__(256) uint8_t g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_workspace_addr[kMaxDevices];
+
+// Device address of g_static_workspace on the current device (looked up with
+// that device current, once), or nullptr on failure.
+void* static_workspace_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = g_static_workspace_addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return nullptr;
+    g_static_workspace_addr[dev].store(p, std::memory_order_release);
+    return p;
+}
+
+}  // namespace
+
+extern "C" pkv_status paged_gqa_decode_attention_static_workspace(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+    int32_t num_blocks, int32_t max_context_len, float softmax_scale, int32_t kv_dtype,
+    float k_scale, float v_scale, int32_t partition_tokens, void* stream) {
+    // Split-KV needs scratch only when more than one partition covers the
+    // longest context (the same rule paged_gqa_decode_attention applies).
+    const bool split = partition_tokens > 0 && partition_tokens < max_context_len;
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    if (split && batch > 0 && num_kv_heads > 0 && num_q_heads > 0 && block_size > 0 &&
+        partition_tokens % block_size == 0) {
+        ws_bytes = paged_gqa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                   max_context_len, partition_tokens);
+        if (ws_bytes > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;
+        if (ws_bytes > 0) {
+            ws = static_workspace_address();
+            if (!ws) return PKV_ERR_CUDA;
+            // the previous call may have left other data where this call's
+            // partition counters go: clear them, in stream order
+            const int32_t P = (partition_tokens + kPageRows - 1) / kPageRows * kPageRows;
+            const int nparts = std::max(1, (max_context_len + P - 1) / P);
+            const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, num_kv_heads, nparts);
+            if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + wl.count, 0,
+                                (size_t)batch * num_kv_heads * sizeof(unsigned int),
+                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            ws_bytes = PKV_STATIC_WORKSPACE_BYTES;
+        }
+    }
+    return paged_gqa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                      num_q_heads, num_kv_heads, head_dim, block_size,
+                                      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                                      kv_dtype, k_scale, v_scale, partition_tokens, ws, ws_bytes,
+                                      stream);
+}
