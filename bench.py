@@ -234,8 +234,11 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="qwen2.5-1.5b", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=-1,
-                    help="split-KV partition tokens (-1: the library's suggestion; 0: single pass)")
+                    help="split-KV plan: -1 the library's balanced plan (default), 0 single pass, "
+                         "P > 0 fixed partitions of P tokens")
     ap.add_argument("--graph-steps", type=int, default=500, help="steps per captured CUDA graph")
+    ap.add_argument("--unfused", action="store_true",
+                    help="two launches per step (cache write, then attention) instead of the fused step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-baseline-s", type=float, default=10.0)
     ap.add_argument("--seed", type=int, default=0)
@@ -296,8 +299,6 @@ def run_ours(args):
     max_len = int(lens.max())
     fp8 = w.kv_dtype == "fp8"
     P = args.partition
-    if P < 0:
-        P = w.partition_tokens or pkv.paged_gqa_decode_suggest_partition(B, Hkv, max_len, bs, 0)
     attn_b, cw_b = step_bytes(w, lens, B)
     step_b = attn_b + cw_b
 
@@ -324,20 +325,29 @@ def run_ours(args):
     else:
         base_k, base_v = k16, v16
     pools = [(base_k, base_v)] + [(base_k.clone(), base_v.clone()) for _ in range(R - 1)]
-    ws_n = pkv.paged_gqa_decode_workspace_size(B, Hq, Hkv, D, max_len, P) if P else 0
+    ws_n = pkv.paged_gqa_decode_workspace_size(B, Hq, Hkv, D, max_len, P)
     ws = torch.zeros(max(ws_n, 256), dtype=torch.uint8, device=device)
     out = torch.empty((B, Hq, D), dtype=torch.float16, device=device)
 
+    fused = not args.unfused and P == pkv.PKV_PARTITION_AUTO
+
     def cache_write(i):
+        if fused:                                  # the step kernel writes the new tokens itself
+            return
         kc, vc = pools[i % R]
         pkv.paged_kv_cache_write(k_new, v_new, kc, vc, slots, kv_dtype=w.kv_dtype, k_scale=ks,
                                  v_scale=vs, stream=stream)
 
     def attention(i):
         kc, vc = pools[i % R]
-        pkv.paged_gqa_decode_attention(out, q, kc, vc, bt, cl, max_context_len=max_len,
-                                       softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
-                                       v_scale=vs, partition_tokens=P, workspace=ws, stream=stream)
+        if fused:
+            pkv.paged_gqa_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, max_context_len=max_len,
+                                      softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
+                                      workspace=ws, stream=stream)
+        else:
+            pkv.paged_gqa_decode_attention(out, q, kc, vc, bt, cl, max_context_len=max_len,
+                                           softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
+                                           v_scale=vs, partition_tokens=P, workspace=ws, stream=stream)
 
     # ---- warm-up: W eager steps (also sets kernel attributes and TMA maps) ----
     for i in range(args.warmup):
@@ -382,7 +392,7 @@ def run_ours(args):
         attn_ms += [a.elapsed_time(b) for a, b in graphs[n][1]]
     elapsed_ms = start.elapsed_time(end)
     elapsed_max = reduce_max(elapsed_ms, world, device)
-    launches = 2 * K
+    launches = (1 if fused else 2) * K
 
     # ---- e2e: the public API on host buffers, copies in the timed region ----
     e2e = None
@@ -399,12 +409,18 @@ def run_ours(args):
             for k in h:
                 d[k].copy_(h[k], non_blocking=True)
             kc, vc = pools[i % R]
-            pkv.paged_kv_cache_write(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"],
-                                     kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs, stream=stream)
-            pkv.paged_gqa_decode_attention(out, d["q"], kc, vc, d["block_tables"], d["context_lens"],
-                                           max_context_len=max_len, softmax_scale=scale,
-                                           kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                           partition_tokens=P, workspace=ws, stream=stream)
+            if fused:
+                pkv.paged_gqa_decode_step(out, d["q"], d["k_new"], d["v_new"], kc, vc, d["block_tables"],
+                                          d["context_lens"], max_context_len=max_len, softmax_scale=scale,
+                                          kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs, workspace=ws,
+                                          stream=stream)
+            else:
+                pkv.paged_kv_cache_write(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"],
+                                         kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs, stream=stream)
+                pkv.paged_gqa_decode_attention(out, d["q"], kc, vc, d["block_tables"], d["context_lens"],
+                                               max_context_len=max_len, softmax_scale=scale,
+                                               kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
+                                               partition_tokens=P, workspace=ws, stream=stream)
             out_h.copy_(out, non_blocking=True)
             stream.synchronize()
 
@@ -426,7 +442,8 @@ def run_ours(args):
         peaks, peak_src = measured_peaks()
         peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
         mean_attn_ms = sum(attn_ms) / len(attn_ms)
-        achieved = attn_b / (mean_attn_ms * 1e-3) / 1e9
+        kern_b = step_b if fused else attn_b          # the fused launch also does the cache write
+        achieved = kern_b / (mean_attn_ms * 1e-3) / 1e9
         traffic = recorded_traffic(w.name, P)
         value = world * step_b * K / (elapsed_max * 1e-3) / 1e9
         line = {
@@ -441,11 +458,14 @@ def run_ours(args):
                        "partition_tokens": P, "parallelism": f"dp{world} (independent batches)",
                        "l2": f"inputs larger than L2: {R} KV pool replicas rotated, "
                              f"{R * touched / 2**20:.0f} MiB touched per cycle",
-                       "timing": f"{len(chunks)} CUDA graph replays of <= {S} steps"},
-            "roofline": {"bound": "hbm", "kernel": "decode_attention_kernel",
+                       "timing": f"{len(chunks)} CUDA graph replays of <= {S} steps",
+                       "step": "one fused launch (cache write + attention)" if fused
+                               else "cache write + attention launches"},
+            "roofline": {"bound": "hbm",
+                         "kernel": "decode_balanced_kernel (fused step)" if fused else "decode attention",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
-                         "traffic": traffic, "algorithmic_bytes_per_launch": attn_b,
+                         "traffic": traffic, "algorithmic_bytes_per_launch": kern_b,
                          "mean_launch_us": mean_attn_ms * 1e3},
             "gpu_launches": launches,
             "clocks": sampler.summary(wall0, wall1),

@@ -81,6 +81,11 @@ typedef enum {
     PKV_KV_FP8_E4M3 = 1        /* uint8 OCP E4M3 cache with per-tensor scales */
 } pkv_kv_dtype;
 
+/* partition_tokens value that lets the library plan the split-KV work: the
+ * load-balanced streaming kernel (every warp of a persistent grid takes an
+ * equal share of the batch's pages, whatever the length mix). */
+#define PKV_PARTITION_AUTO (-1)
+
 /* Bits of the device error word (pkv_device_error). */
 #define PKV_DEVERR_CONTEXT_LEN   0x1u  /* a context length exceeded max_context_len or the
                                           table capacity; it was clamped */
@@ -115,9 +120,11 @@ pkv_status paged_kv_cache_write(const void* k_new, const void* v_new,
 
 /*
  * Bytes of workspace paged_gqa_decode_attention needs for these sizes:
- * 0 when partition_tokens == 0 (single pass), else partial results of
- * ceil(max_context_len / partition_tokens) partitions per (sequence, query
- * head) plus one counter per (sequence, KV head). Returns 0 for invalid sizes.
+ * 0 when partition_tokens == 0 (single pass); for partition_tokens > 0 the
+ * partial results of ceil(max_context_len / partition_tokens) partitions per
+ * (sequence, query head) plus one counter per (sequence, KV head); for
+ * PKV_PARTITION_AUTO two partial results per worker warp of the persistent
+ * grid on the CURRENT device plus the counters. Returns 0 for invalid sizes.
  */
 size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads,
                                        int32_t num_kv_heads, int32_t head_dim,
@@ -143,6 +150,13 @@ int32_t paged_gqa_decode_suggest_partition(int32_t batch, int32_t num_kv_heads,
  * where K_t = k_cache[block_tables[b][t / bs]][t % bs][g] (times k_scale for
  * FP8) and likewise V_t. L == 0 gives an all-zero row. Accumulation is fp32.
  *
+ * partition_tokens == PKV_PARTITION_AUTO: the library's plan, normally the
+ *   load-balanced streaming kernel: a persistent grid whose worker warps each
+ *   take an equal contiguous share of all (sequence, KV head, page) units;
+ *   pieces of a (sequence, KV head) split between workers are merged by the
+ *   log-sum-exp rule below by the last piece to finish. Batches above 8192
+ *   sequences fall back to fixed partitions of
+ *   paged_gqa_decode_suggest_partition(...) tokens.
  * partition_tokens == 0: one pass per (sequence, KV head).
  * partition_tokens  > 0: a multiple of block_size; tokens [p*P, (p+1)*P) form
  *   partition p, each partition computes its own (max, sum, output) and the
@@ -170,6 +184,33 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q,
                                       int32_t partition_tokens,
                                       void* workspace, size_t workspace_bytes,
                                       void* stream);
+
+/*
+ * paged_gqa_decode_step -- one decode step in one launch: this step's token
+ * of every sequence is written into the cache and attended to.
+ *
+ * For each b with L = context_lens[b] > 0, the token at position L - 1 (the
+ * context length counts it) is the new one: its K/V, k_new[b] and v_new[b]
+ * ([B, Hkv, D] f16), are stored at slot block_tables[b][(L-1)/bs]*bs + (L-1)%bs
+ * exactly as paged_kv_cache_write stores them (FP8: the same E4M3 codes),
+ * and out is what paged_gqa_decode_attention computes on the updated cache.
+ * The pages motivate the fusion: the engine's fused kernels and graph replay
+ * exist to cut per-step launches ("rvLLM 소개", §CUDA 그래프 리플레이 and
+ * §퓨즈드 CUDA 커널); the kernel that reads the new token's page patches the
+ * row in shared memory and writes it to the cache, so no second launch is
+ * needed. Always the load-balanced plan: `workspace` as for
+ * paged_gqa_decode_attention with PKV_PARTITION_AUTO (zero-filled before its
+ * first use). Batches above 8192 sequences return PKV_ERR_UNSUPPORTED.
+ */
+pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
+                                 void* k_cache, void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int32_t num_blocks,
+                                 int32_t max_context_len, float softmax_scale,
+                                 int32_t kv_dtype, float k_scale, float v_scale,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static text for a status code. Never NULL. */
 const char* pkv_status_string(pkv_status status);

@@ -31,6 +31,8 @@ _SIGNATURES = {
     "paged_gqa_decode_suggest_partition": ([_i32, _i32, _i32, _i32, _i32], _i32),
     "paged_gqa_decode_attention": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                     _i32, _f32, _i32, _f32, _f32, _i32, _P, _sz, _P], ctypes.c_int),
+    "paged_gqa_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                               _i32, _f32, _i32, _f32, _f32, _P, _sz, _P], ctypes.c_int),
     "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "pkv_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
     "paged_gqa_decode_attention_static_workspace": (
@@ -68,6 +70,7 @@ def __getattr__(name):
 
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_WORKSPACE, PKV_ERR_CUDA = range(5)
 PKV_KV_F16, PKV_KV_FP8_E4M3 = 0, 1
+PKV_PARTITION_AUTO = -1         # partition_tokens: the library's load-balanced plan
 DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 _KV_DTYPES = {"f16": PKV_KV_F16, "fp8": PKV_KV_FP8_E4M3}
 
@@ -164,6 +167,33 @@ def paged_gqa_decode_attention(out, q, k_cache, v_cache, block_tables, context_l
         B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(softmax_scale),
         kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), int(partition_tokens),
         _ptr(workspace), ws_bytes, _stream(stream)), "paged_gqa_decode_attention")
+
+
+def paged_gqa_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, *,
+                          max_context_len, softmax_scale, kv_dtype="f16", k_scale=1.0, v_scale=1.0,
+                          workspace=None, stream=None) -> None:
+    """One decode step in one launch: k_new/v_new [B, Hkv, D] go to position
+    context_lens[b] - 1 of each sequence's pages, then out = attention over the
+    updated cache (the load-balanced plan; workspace sized for PKV_PARTITION_AUTO)."""
+    cdt = "uint8" if kv_dtype == "fp8" else "float16"
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    _dense("k_new", k_new, "float16")
+    _dense("v_new", v_new, "float16")
+    _dense("k_cache", k_cache, cdt)
+    _dense("v_cache", v_cache, cdt)
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    if workspace is not None:
+        _dense("workspace", workspace, "uint8", "float32", "int32")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load_library().paged_gqa_decode_step(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
+        float(softmax_scale), kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _ptr(workspace),
+        ws_bytes, _stream(stream)), "paged_gqa_decode_step")
 
 
 def pkv_device_error() -> int:

@@ -52,6 +52,8 @@ __device__ __forceinline__ uint2 quantize8_e4m3(uint4 x, float scale) {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t total = static_cast<int64_t>(p.num_tokens) * p.chunks_per_token;
     if (idx >= total) return;

@@ -33,13 +33,9 @@
 // folded into the logit scale and v_scale into the output.
 #pragma once
 
-#include "pkv_device.cuh"
+#include "decode_page.cuh"
 
 namespace pkv {
-
-constexpr int kHeadDim = 128;
-constexpr int kPageRows = 16;   // block_size
-constexpr int kGroupPad = 8;    // query heads per KV head, padded to the mma N
 
 struct DecodeParams {
     __half* out;                  // [B, Hq, D]
@@ -87,6 +83,8 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
 
+    grid_dependency_wait();                      // inputs may come from the previous launch
+    grid_dependents_launch();
     // ---- this CTA's token range (uniform across the CTA) ----
     int L = __ldg(p.context_lens + b);
     const int cap = min(p.max_context_len, p.max_blocks_per_seq * kPageRows);
@@ -182,28 +180,11 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
 
     // ================================ consumers ================================
     const int r = lane >> 2, c = lane & 3;      // fragment row group / column pair
-    // Q^T as the B operand (16 channels x 8 heads per k-step); head r of g.
     uint32_t qf[8][2];
-    {
-        const bool live = r < G;
-        const uint32_t* qh = reinterpret_cast<const uint32_t*>(
-            p.q + ((int64_t)b * p.Hq + (int64_t)g * G + (live ? r : 0)) * kHeadDim);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            // f16 cache: channels 16j+2c(+1) and 16j+8+2c(+1);
-            // FP8 cache: channels 16j+4c(+1) and 16j+4c+2(+1), matching the byte tile fragments.
-            const int d0 = kFp8 ? 16 * j + 4 * c : 16 * j + 2 * c;
-            const int d1 = kFp8 ? d0 + 2 : d0 + 8;
-            qf[j][0] = live ? __ldg(qh + d0 / 2) : 0u;
-            qf[j][1] = live ? __ldg(qh + d1 / 2) : 0u;
-        }
-    }
-    const float sl = p.logit_scale_log2;
-    float m0 = -INFINITY, m1 = -INFINITY;      // running max of heads 2c, 2c+1
-    float l0 = 0.f, l1 = 0.f;                  // this lane's share of the running sums
-    float o[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    load_q_fragments<kFp8>(
+        qf, r < G ? p.q + ((int64_t)b * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, c);
+    WarpState st;
+    st.reset();
 
     for (int it = 0; it < n_iters; ++it) {
         const int s = it % kStages;
@@ -214,116 +195,14 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int blk = it * kConsumers + warp;
         if (blk < nblk) {
             const int valid = blk == nblk - 1 ? last_valid : kPageRows;
-            const uint32_t kt = k_tile(s, warp), vt = v_tile(s, warp);
-
-            // ---- S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T ----
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (!kFp8) {
-                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const int chunk = (kk & 3) * 2 + (lane >> 4);
-                    const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(addr, a0, a1, a2, a3);
-                    mma_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-                }
-            } else {
-                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-                for (int J = 0; J < 4; ++J) {
-                    const int chunk = 2 * J + (lane >> 4);
-                    const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
-                    uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
-                    ldsm_x4(addr, r0, r1, r2, r3);
-                    mma_16816(sacc, e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
-                              e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
-                              qf[2 * J][0], qf[2 * J][1]);
-                    mma_16816(sacc, e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
-                              e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
-                              qf[2 * J + 1][0], qf[2 * J + 1][1]);
-                }
-            }
-
-            // ---- online softmax over this block's tokens (rows r, r+8) ----
-            float x0 = sacc[0] * sl, x1 = sacc[1] * sl, x2 = sacc[2] * sl, x3 = sacc[3] * sl;
-            if (valid < kPageRows) {                // rows past the context: excluded
-                if (r >= valid) x0 = x1 = -INFINITY;
-                if (r + 8 >= valid) x2 = x3 = -INFINITY;
-            }
-            float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-                bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-            }
-            const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-            const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-            m0 = mn0;
-            m1 = mn1;
-            const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
-            const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
-            l0 = l0 * al0 + (p0 + p2);
-            l1 = l1 * al1 + (p1 + p3);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
-            }
-            // P^T as the B operand: transpose the (token x head) accumulator layout.
-            const uint32_t pb0 = movmatrix_trans(pack_half2(p0, p1));   // tokens 0..7
-            const uint32_t pb1 = movmatrix_trans(pack_half2(p2, p3));   // tokens 8..15
-
-            // ---- O^T (128 ch x 8 heads) += V^T (128 x 16 tokens) . P^T ----
-            if constexpr (!kFp8) {
-                uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // zero V of excluded rows
-                if (valid < kPageRows) {
-                    mlo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
-                    mhi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
-                }
-                const int row = (lane & 7) + (lane >> 4) * 8;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int chunk = (i & 3) * 2 + ((lane >> 3) & 1);
-                    const uint32_t addr = vt + (i >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_trans(addr, a0, a1, a2, a3);
-                    mma_16816(o[i], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
-                }
-            } else {
-                // lane (r, c) reads channels 16r..16r+15 of token rows 2c, 2c+1, 2c+8, 2c+9
-                auto row_addr = [&](int t) { return vt + t * 128 + ((r ^ (t & 7)) << 4); };
-                uint4 va = lds128(row_addr(2 * c)), vb = lds128(row_addr(2 * c + 1));
-                uint4 vc = lds128(row_addr(2 * c + 8)), vd = lds128(row_addr(2 * c + 9));
-                if (valid < kPageRows) {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    if (2 * c >= valid) va = z;
-                    if (2 * c + 1 >= valid) vb = z;
-                    if (2 * c + 8 >= valid) vc = z;
-                    if (2 * c + 9 >= valid) vd = z;
-                }
-                const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-                const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
-                // m-tile i: rows r / r+8 are channels 16r+2i / 16r+2i+1 (bytes 2(i%2), +1 of word i/2)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t sel = (i & 1) ? 0x7362u : 0x5140u;
-                    const uint32_t top = prmt(wa[i >> 1], wb[i >> 1], sel);   // tokens 2c, 2c+1
-                    const uint32_t bot = prmt(wc[i >> 1], wd[i >> 1], sel);   // tokens 2c+8, 2c+9
-                    mma_16816(o[i], e4m3x2_to_half2(top), e4m3x2_to_half2(top >> 16),
-                              e4m3x2_to_half2(bot), e4m3x2_to_half2(bot >> 16), pb0, pb1);
-                }
-            }
+            attend_page<kFp8>(st, k_tile(s, warp), v_tile(s, warp), valid, qf, p.logit_scale_log2, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(s));
     }
 
     // ---- merge the consumer warps through shared memory (ring reused) ----
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
+    st.reduce_l();
     constexpr int kCT = 32 * kConsumers;
     consumer_sync(kCT);                           // every warp is done with the ring
     float* red_o = reinterpret_cast<float*>(ring_ptr);                 // [warp][head][D]
@@ -333,18 +212,17 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
         float* ow = red_o + warp * kGroupPad * kHeadDim;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int d_lo = kFp8 ? 16 * r + 2 * i : 16 * i + r;
-            const int d_hi = kFp8 ? d_lo + 1 : d_lo + 8;
-            ow[(2 * c) * kHeadDim + d_lo] = o[i][0];
-            ow[(2 * c + 1) * kHeadDim + d_lo] = o[i][1];
-            ow[(2 * c) * kHeadDim + d_hi] = o[i][2];
-            ow[(2 * c + 1) * kHeadDim + d_hi] = o[i][3];
+            const int d_lo = out_channel_lo<kFp8>(r, i), d_hi = out_channel_hi<kFp8>(r, i);
+            ow[(2 * c) * kHeadDim + d_lo] = st.o[i][0];
+            ow[(2 * c + 1) * kHeadDim + d_lo] = st.o[i][1];
+            ow[(2 * c) * kHeadDim + d_hi] = st.o[i][2];
+            ow[(2 * c + 1) * kHeadDim + d_hi] = st.o[i][3];
         }
         if (r == 0) {
-            red_m[warp * kGroupPad + 2 * c] = m0;
-            red_m[warp * kGroupPad + 2 * c + 1] = m1;
-            red_l[warp * kGroupPad + 2 * c] = l0;
-            red_l[warp * kGroupPad + 2 * c + 1] = l1;
+            red_m[warp * kGroupPad + 2 * c] = st.m0;
+            red_m[warp * kGroupPad + 2 * c + 1] = st.m1;
+            red_l[warp * kGroupPad + 2 * c] = st.l0;
+            red_l[warp * kGroupPad + 2 * c + 1] = st.l1;
         }
     }
     consumer_sync(kCT);
@@ -386,17 +264,61 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
     consumer_sync(kCT);
     if (!s_is_last) return;
     __threadfence();
-    for (int h = h_first; h < G; h += h_step) {
-        const int64_t pr0 = (row0 + h) * p.nparts;
-        float M = -INFINITY;
-        for (int q = 0; q < nparts_b; ++q) M = fmaxf(M, __ldcg(p.ws_m + pr0 + q));
-        float wsum = 0.f, acc = 0.f;
-        for (int q = 0; q < nparts_b; ++q) {
-            const float w = __ldcg(p.ws_l + pr0 + q) * fast_exp2(__ldcg(p.ws_m + pr0 + q) - M);
-            wsum += w;
-            acc += w * __ldcg(p.ws_o + (pr0 + q) * kHeadDim + d);
+    // weights w_q = l_q * exp2(m_q - M) of every partition and head, staged in
+    // shared memory (the ring is free), then one pass over the outputs
+    float* wts = reinterpret_cast<float*>(ring_ptr);             // [G][nparts_b]
+    const bool staged = (size_t)G * nparts_b * sizeof(float) <= (size_t)S::kRingBytes;
+    if (staged) {
+        for (int i = threadIdx.x; i < G * nparts_b; i += kCT) {
+            const int h = i / nparts_b, q = i - h * nparts_b;
+            wts[i] = __ldcg(p.ws_m + (row0 + h) * p.nparts + q);
         }
-        out_g[h * kHeadDim + d] = __float2half_rn(acc / wsum * p.out_scale);
+        consumer_sync(kCT);
+        // one warp per head: max, weights, normaliser
+        for (int h = warp; h < G; h += kConsumers) {
+            float* wh = wts + h * nparts_b;
+            float M = -INFINITY;
+            for (int q = lane; q < nparts_b; q += 32) M = fmaxf(M, wh[q]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            float sum = 0.f;
+            for (int q = lane; q < nparts_b; q += 32) {
+                const float w = __ldcg(p.ws_l + (row0 + h) * p.nparts + q) * fast_exp2(wh[q] - M);
+                wh[q] = w;
+                sum += w;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            __syncwarp();
+            for (int q = lane; q < nparts_b; q += 32) wh[q] *= p.out_scale / sum;
+        }
+        consumer_sync(kCT);
+        for (int h = h_first; h < G; h += h_step) {
+            const float* wh = wts + h * nparts_b;
+            const float* src = p.ws_o + (row0 + h) * p.nparts * kHeadDim + d;
+            float acc = 0.f;
+            int q = 0;
+            for (; q + 4 <= nparts_b; q += 4) {
+                const float v0 = __ldcg(src + (q + 0) * kHeadDim), v1 = __ldcg(src + (q + 1) * kHeadDim);
+                const float v2 = __ldcg(src + (q + 2) * kHeadDim), v3 = __ldcg(src + (q + 3) * kHeadDim);
+                acc += wh[q] * v0 + wh[q + 1] * v1 + wh[q + 2] * v2 + wh[q + 3] * v3;
+            }
+            for (; q < nparts_b; ++q) acc += wh[q] * __ldcg(src + q * kHeadDim);
+            out_g[h * kHeadDim + d] = __float2half_rn(acc);
+        }
+    } else {
+        for (int h = h_first; h < G; h += h_step) {
+            const int64_t pr0 = (row0 + h) * p.nparts;
+            float M = -INFINITY;
+            for (int q = 0; q < nparts_b; ++q) M = fmaxf(M, __ldcg(p.ws_m + pr0 + q));
+            float wsum = 0.f, acc = 0.f;
+            for (int q = 0; q < nparts_b; ++q) {
+                const float w = __ldcg(p.ws_l + pr0 + q) * fast_exp2(__ldcg(p.ws_m + pr0 + q) - M);
+                wsum += w;
+                acc += w * __ldcg(p.ws_o + (pr0 + q) * kHeadDim + d);
+            }
+            out_g[h * kHeadDim + d] = __float2half_rn(acc / wsum * p.out_scale);
+        }
     }
     if (threadIdx.x == 0) p.ws_count[(int64_t)b * p.Hkv + g] = 0u;   // ready for the next call
 }

@@ -1,0 +1,178 @@
+// Per-warp building blocks of paged GQA decode attention: the query-group
+// fragments, and the online-softmax update of one 16-token page of K/V held in
+// shared memory (a 128-byte-swizzled TMA tile).
+//
+// Layout of the tensor-core work (mma.sync m16n8k16, f16 in, f32 accumulate),
+// chosen so that the KV tokens sit on the M side and the G <= 8 query heads of
+// one KV head on N = 8 (G = 6 or 7 for Qwen2.5 wastes 1/4 or 1/8 of N, where
+// putting the heads on M = 16 would waste 5/8):
+//   S^T (16 tok x 8 heads) = K (16 tok x 128 ch) . Q^T (128 ch x 8 heads)
+//   O^T (128 ch x 8 heads) += V^T (128 ch x 16 tok) . P^T (16 tok x 8 heads)
+// Lane (r, c) = (lane / 4, lane % 4) holds the logits of tokens r, r+8 for
+// heads 2c, 2c+1 and the output of the same two heads, so the softmax rescale
+// is lane-local; P^T reaches the B-operand layout by an 8x8 transpose
+// (movmatrix). The contraction over channels may use any channel order as long
+// as K and Q agree; the FP8 path uses that freedom to read 4 codes per lane.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int kHeadDim = 128;
+constexpr int kPageRows = 16;   // block_size
+constexpr int kGroupPad = 8;    // query heads per KV head, padded to the mma N
+
+// Running softmax state of one warp over the tokens it has seen.
+struct WarpState {
+    float m0, m1;       // running max (exp2 domain) of heads 2c, 2c+1
+    float l0, l1;       // this lane's share of the running sums
+    float o[8][4];      // O^T fragments: m-tile i, rows r / r+8, heads 2c / 2c+1
+
+    __device__ __forceinline__ void reset() {
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    }
+    // Sums the lanes' shares of l over the 8 lanes that hold the same heads.
+    __device__ __forceinline__ void reduce_l() {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        }
+    }
+};
+
+// Channel held by lane (r, c) in m-tile i of O^T, rows r and r+8.
+template <bool kFp8>
+__device__ __forceinline__ int out_channel_lo(int r, int i) { return kFp8 ? 16 * r + 2 * i : 16 * i + r; }
+template <bool kFp8>
+__device__ __forceinline__ int out_channel_hi(int r, int i) { return kFp8 ? 16 * r + 2 * i + 1 : 16 * i + r + 8; }
+
+// Q^T as the B operand for the query head of row r (16 channels per k-step);
+// `qrow` is that head's 128 f16 channels, or nullptr for a padding head.
+template <bool kFp8>
+__device__ __forceinline__ void load_q_fragments(uint32_t (&qf)[8][2], const __half* qrow, int c) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        // f16 cache: channels 16j+2c(+1) and 16j+8+2c(+1);
+        // FP8 cache: channels 16j+4c(+1) and 16j+4c+2(+1), matching the byte tile fragments.
+        const int d0 = kFp8 ? 16 * j + 4 * c : 16 * j + 2 * c;
+        const int d1 = kFp8 ? d0 + 2 : d0 + 8;
+        qf[j][0] = qrow ? __ldg(q32 + d0 / 2) : 0u;
+        qf[j][1] = qrow ? __ldg(q32 + d1 / 2) : 0u;
+    }
+}
+
+// Online-softmax update of `st` with one page: K tile at shared address kt, V
+// tile at vt (f16: two 2 KiB boxes of 64 channels each; FP8: one 2 KiB box),
+// the first `valid` rows live. `sl` = softmax scale * log2(e) (* k_scale).
+template <bool kFp8>
+__device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t vt, int valid,
+                                            const uint32_t (&qf)[8][2], float sl, int lane) {
+    const int r = lane >> 2, c = lane & 3;
+
+    // ---- S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T ----
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+        if constexpr (!kFp8) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int chunk = (kk & 3) * 2 + (lane >> 4);
+                const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(addr, a0, a1, a2, a3);
+                mma_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+            }
+        } else {
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                const int chunk = 2 * J + (lane >> 4);
+                const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
+                uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
+                ldsm_x4(addr, r0, r1, r2, r3);
+                mma_16816(sacc, e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
+                          e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
+                          qf[2 * J][0], qf[2 * J][1]);
+                mma_16816(sacc, e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
+                          e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
+                          qf[2 * J + 1][0], qf[2 * J + 1][1]);
+            }
+        }
+    }
+
+    // ---- online softmax over this page's tokens (rows r, r+8) ----
+    float x0 = sacc[0] * sl, x1 = sacc[1] * sl, x2 = sacc[2] * sl, x3 = sacc[3] * sl;
+    if (valid < kPageRows) {                    // rows past the context: excluded
+        if (r >= valid) x0 = x1 = -INFINITY;
+        if (r + 8 >= valid) x2 = x3 = -INFINITY;
+    }
+    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+    }
+    const float mn0 = fmaxf(st.m0, bm0), mn1 = fmaxf(st.m1, bm1);
+    const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
+    st.m0 = mn0;
+    st.m1 = mn1;
+    const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
+    const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+    st.l0 = st.l0 * al0 + (p0 + p2);
+    st.l1 = st.l1 * al1 + (p1 + p3);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        st.o[i][0] *= al0; st.o[i][1] *= al1; st.o[i][2] *= al0; st.o[i][3] *= al1;
+    }
+    // P^T as the B operand: transpose the (token x head) accumulator layout.
+    const uint32_t pb0 = movmatrix_trans(pack_half2(p0, p1));   // tokens 0..7
+    const uint32_t pb1 = movmatrix_trans(pack_half2(p2, p3));   // tokens 8..15
+
+    // ---- O^T (128 ch x 8 heads) += V^T (128 x 16 tokens) . P^T ----
+    if constexpr (!kFp8) {
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // zero V of excluded rows
+        if (valid < kPageRows) {
+            mlo = (2 * c < valid ? 0x0000ffffu : 0u) | (2 * c + 1 < valid ? 0xffff0000u : 0u);
+            mhi = (2 * c + 8 < valid ? 0x0000ffffu : 0u) | (2 * c + 9 < valid ? 0xffff0000u : 0u);
+        }
+        const int row = (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int chunk = (i & 3) * 2 + ((lane >> 3) & 1);
+            const uint32_t addr = vt + (i >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_trans(addr, a0, a1, a2, a3);
+            mma_16816(st.o[i], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
+        }
+    } else {
+        // lane (r, c) reads channels 16r..16r+15 of token rows 2c, 2c+1, 2c+8, 2c+9
+        auto row_addr = [&](int t) { return vt + t * 128 + ((r ^ (t & 7)) << 4); };
+        uint4 va = lds128(row_addr(2 * c)), vb = lds128(row_addr(2 * c + 1));
+        uint4 vc = lds128(row_addr(2 * c + 8)), vd = lds128(row_addr(2 * c + 9));
+        if (valid < kPageRows) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            if (2 * c >= valid) va = z;
+            if (2 * c + 1 >= valid) vb = z;
+            if (2 * c + 8 >= valid) vc = z;
+            if (2 * c + 9 >= valid) vd = z;
+        }
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+        const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+        // m-tile i: rows r / r+8 are channels 16r+2i / 16r+2i+1 (bytes 2(i%2), +1 of word i/2)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t sel = (i & 1) ? 0x7362u : 0x5140u;
+            const uint32_t top = prmt(wa[i >> 1], wb[i >> 1], sel);   // tokens 2c, 2c+1
+            const uint32_t bot = prmt(wc[i >> 1], wd[i >> 1], sel);   // tokens 2c+8, 2c+9
+            mma_16816(st.o[i], e4m3x2_to_half2(top), e4m3x2_to_half2(top >> 16),
+                      e4m3x2_to_half2(bot), e4m3x2_to_half2(bot >> 16), pb0, pb1);
+        }
+    }
+}
+
+}  // namespace pkv

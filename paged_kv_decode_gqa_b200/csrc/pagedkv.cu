@@ -15,6 +15,7 @@
 #include "pagedkv.h"
 #include "cache_write.cuh"
 #include "decode_attention.cuh"
+#include "decode_balanced.cuh"
 
 namespace {
 
@@ -24,6 +25,14 @@ using pkv::kPageRows;
 constexpr int kConsumers = 4;
 constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
 constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
+
+// Balanced streaming kernel: 4 worker warps per CTA, each with its own ring
+// of page slots (f16: 3 x 8 KiB, FP8: 6 x 4 KiB), two CTAs per SM.
+constexpr int kBalWarps = 4;
+constexpr int kBalStagesF16 = 3;
+constexpr int kBalStagesFp8 = 6;
+constexpr int kBalMaxBatch = 8192;        // unit-order tables must fit in shared memory
+constexpr int kBalMinUnits = 4;           // pages per worker at least (small batches)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -91,6 +100,25 @@ bool cached_cache_map(CUtensorMap* out, const void* base, bool fp8, int num_bloc
     return true;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous launch in the stream finishes; it waits (griddepcontrol.wait)
+// before its first global-memory access.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Opt a kernel into its dynamic shared memory once per device.
 template <typename Kernel>
 cudaError_t ensure_smem(Kernel kernel, int bytes, unsigned long long* done_mask) {
@@ -112,13 +140,115 @@ pkv_status launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& mk, co
     static unsigned long long done = 0;
     if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
     dim3 grid(prm.nparts, Hkv, B);
-    kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(mk, mv, prm);
-    return cudaPeekAtLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mk, mv, prm) == cudaSuccess
+               ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <bool kFp8>
+using BalShape = pkv::BalancedShape<kFp8, kBalWarps, kFp8 ? kBalStagesFp8 : kBalStagesF16>;
+
+template <bool kFp8, bool kFuse = false>
+auto balanced_kernel() {
+    return pkv::decode_balanced_kernel<kFp8, kBalWarps, kFp8 ? kBalStagesFp8 : kBalStagesF16, kFuse>;
+}
+
+// Persistent grid of the balanced kernel for batch B on the current device:
+// as many CTAs as fit at once (0 on error). Both the plain and the fused
+// variant are opted into their shared memory here.
+template <bool kFp8>
+int balanced_grid(int B) {
+    static unsigned long long done = 0, done_fused = 0;
+    auto kernel = balanced_kernel<kFp8>();
+    if (ensure_smem(balanced_kernel<kFp8, true>(), (int)BalShape<kFp8>::smem_bytes(kBalMaxBatch),
+                    &done_fused) != cudaSuccess)
+        return 0;
+    if (ensure_smem(kernel, (int)BalShape<kFp8>::smem_bytes(kBalMaxBatch), &done) != cudaSuccess) return 0;
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, BalShape<kFp8>::kThreads,
+                                                      BalShape<kFp8>::smem_bytes(B)) != cudaSuccess)
+        return 0;
+    return std::max(1, per_sm) * sms;
+}
+
+struct BalancedLayout {
+    size_t o, ml, count, total;
+};
+
+BalancedLayout balanced_layout(int64_t workers, int64_t B, int64_t Hkv) {
+    BalancedLayout w{};
+    w.o = 0;
+    w.ml = align256(2 * workers * 32 * 8 * sizeof(float4));
+    w.count = w.ml + align256(2 * workers * 4 * sizeof(float4));
+    w.total = w.count + align256(pkv::kMergeLevels * 2 * workers * sizeof(unsigned int));
+    (void)B;
+    (void)Hkv;
+    return w;
+}
+
+// The balanced kernel serves AUTO unless the batch is too large for its tables.
+bool use_balanced(int64_t B, int64_t Hkv, int64_t max_blocks_per_seq) {
+    return B <= kBalMaxBatch && B * Hkv * max_blocks_per_seq < (int64_t(1) << 31);
 }
 
 struct WorkspaceLayout {
     size_t o, m, l, count, total;
 };
+
+// Launches the balanced kernel (fused with this step's cache write when
+// k_new/v_new are given) after the workspace check.
+pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_new, void* out,
+                           const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                           int32_t Hq, int32_t Hkv, int32_t max_blocks_per_seq, int32_t num_blocks,
+                           int32_t max_context_len, float softmax_scale, float k_scale, float v_scale,
+                           void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    const BalancedLayout bl = balanced_layout((int64_t)grid * kBalWarps, batch, Hkv);
+    if (!workspace || workspace_bytes < bl.total) return PKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    pkv::BalancedParams bp{};
+    bp.out = static_cast<__half*>(out);
+    bp.q = static_cast<const __half*>(q);
+    bp.block_tables = block_tables;
+    bp.context_lens = context_lens;
+    bp.ws_o = reinterpret_cast<float4*>(ws + bl.o);
+    bp.ws_ml = reinterpret_cast<float4*>(ws + bl.ml);
+    bp.ws_count = reinterpret_cast<unsigned int*>(ws + bl.count);
+    bp.k_new = static_cast<const __half*>(k_new);
+    bp.v_new = static_cast<const __half*>(v_new);
+    bp.k_cache = const_cast<void*>(k_cache);
+    bp.v_cache = const_cast<void*>(v_cache);
+    bp.k_scale = k_scale;
+    bp.v_scale = v_scale;
+    bp.B = batch;
+    bp.Hq = Hq;
+    bp.Hkv = Hkv;
+    bp.G = Hq / Hkv;
+    bp.max_blocks_per_seq = max_blocks_per_seq;
+    bp.num_blocks = num_blocks;
+    bp.max_context_len = max_context_len;
+    bp.min_units_per_worker = kBalMinUnits;
+    const float log2e = 1.4426950408889634f;
+    bp.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
+    bp.out_scale = fp8 ? v_scale : 1.f;
+    CUtensorMap mk, mv;
+    if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, Hkv) ||
+        !cached_cache_map(&mv, v_cache, fp8, num_blocks, Hkv))
+        return PKV_ERR_CUDA;
+    const bool fuse = k_new != nullptr;
+    const dim3 g(grid), blk(BalShape<false>::kThreads);
+    cudaError_t e;
+    if (fp8)
+        e = fuse ? launch_pdl(balanced_kernel<true, true>(), g, blk, BalShape<true>::smem_bytes(batch), st, mk, mv, bp)
+                 : launch_pdl(balanced_kernel<true, false>(), g, blk, BalShape<true>::smem_bytes(batch), st, mk, mv, bp);
+    else
+        e = fuse ? launch_pdl(balanced_kernel<false, true>(), g, blk, BalShape<false>::smem_bytes(batch), st, mk, mv, bp)
+                 : launch_pdl(balanced_kernel<false, false>(), g, blk, BalShape<false>::smem_bytes(batch), st, mk, mv, bp);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
 
 WorkspaceLayout workspace_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t nparts) {
     WorkspaceLayout w{};
@@ -129,6 +259,37 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t npa
     w.count = w.l + align256(rows * sizeof(float));
     w.total = w.count + align256(B * Hkv * sizeof(unsigned int));
     return w;
+}
+
+// Host-side argument checks shared by the attention entry points (PKV_OK for
+// a valid call, also when batch == 0).
+pkv_status check_attention_args(const void* out, const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                                int32_t max_context_len, float softmax_scale, int32_t kv_dtype,
+                                float k_scale, float v_scale, int32_t partition_tokens) {
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
+        partition_tokens < PKV_PARTITION_AUTO)
+        return PKV_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return PKV_ERR_INVALID_ARG;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != kHeadDim || block_size != kPageRows) return PKV_ERR_UNSUPPORTED;
+    if (num_q_heads / num_kv_heads > pkv::kGroupPad) return PKV_ERR_UNSUPPORTED;
+    if (partition_tokens > 0 && partition_tokens % block_size != 0) return PKV_ERR_INVALID_ARG;
+    if (batch == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PKV_ERR_INVALID_ARG;
+    if (batch > 65535 || num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
+    return PKV_OK;
 }
 
 }  // namespace
@@ -188,19 +349,28 @@ pkv_status paged_kv_cache_write(const void* k_new, const void* v_new, void* k_ca
     const int64_t blocks = (total + threads - 1) / threads;
     if (blocks > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (fp8)
-        pkv::cache_write_kernel<true><<<(unsigned)blocks, threads, 0, st>>>(prm);
-    else
-        pkv::cache_write_kernel<false><<<(unsigned)blocks, threads, 0, st>>>(prm);
-    return cudaPeekAtLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    const cudaError_t e =
+        fp8 ? launch_pdl(pkv::cache_write_kernel<true>, dim3((unsigned)blocks), dim3(threads), 0, st, prm)
+            : launch_pdl(pkv::cache_write_kernel<false>, dim3((unsigned)blocks), dim3(threads), 0, st, prm);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                        int32_t head_dim, int32_t max_context_len,
                                        int32_t partition_tokens) {
     if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim ||
-        max_context_len < 0 || partition_tokens < 0)
+        max_context_len < 0 || partition_tokens < PKV_PARTITION_AUTO)
         return 0;
+    if (partition_tokens == PKV_PARTITION_AUTO) {
+        const int64_t max_blocks = std::max(1, (max_context_len + kPageRows - 1) / kPageRows);
+        if (use_balanced(batch, num_kv_heads, max_blocks)) {
+            const int grid = std::max(balanced_grid<false>(batch), balanced_grid<true>(batch));
+            if (grid <= 0) return 0;
+            return balanced_layout((int64_t)grid * kBalWarps, batch, num_kv_heads).total;
+        }
+        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
+                                                              kPageRows, 0);
+    }
     if (partition_tokens == 0) return 0;
     const int64_t nparts = std::max<int64_t>(1, (max_context_len + partition_tokens - 1) / partition_tokens);
     return workspace_layout(batch, num_q_heads, num_kv_heads, nparts).total;
@@ -235,26 +405,31 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
                                       int32_t kv_dtype, float k_scale, float v_scale,
                                       int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                       void* stream) {
-    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 || partition_tokens < 0)
-        return PKV_ERR_INVALID_ARG;
-    if (num_q_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
-    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale)) return PKV_ERR_INVALID_ARG;
+    {
+        const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                                  num_q_heads, num_kv_heads, head_dim, block_size,
+                                                  max_blocks_per_seq, num_blocks, max_context_len,
+                                                  softmax_scale, kv_dtype, k_scale, v_scale,
+                                                  partition_tokens);
+        if (v != PKV_OK || batch == 0) return v;
+    }
     const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
-    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
-        return PKV_ERR_INVALID_ARG;
-    if (head_dim != kHeadDim || block_size != kPageRows) return PKV_ERR_UNSUPPORTED;
     const int G = num_q_heads / num_kv_heads;
-    if (G > pkv::kGroupPad) return PKV_ERR_UNSUPPORTED;
-    if (partition_tokens % block_size != 0) return PKV_ERR_INVALID_ARG;
-    if (batch == 0) return PKV_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
-        return PKV_ERR_INVALID_ARG;
-    if (batch > 65535 || num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
+
+    const float log2e = 1.4426950408889634f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (partition_tokens == PKV_PARTITION_AUTO) {
+        if (use_balanced(batch, num_kv_heads, max_blocks_per_seq)) {
+            const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+            if (grid <= 0) return PKV_ERR_CUDA;
+            return launch_balanced(fp8, grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
+                                   context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
+                                   num_blocks, max_context_len, softmax_scale, k_scale, v_scale,
+                                   workspace, workspace_bytes, st);
+        }
+        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
+                                                              kPageRows, 0);
+    }
 
     // plan: a partition covering the longest context is a single pass
     int32_t P = partition_tokens;
@@ -285,7 +460,6 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
     prm.max_context_len = max_context_len;
     prm.partition_tokens = P;
     prm.nparts = nparts;
-    const float log2e = 1.4426950408889634f;
     prm.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
     prm.out_scale = fp8 ? v_scale : 1.f;
 
@@ -293,9 +467,31 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
     if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
         return PKV_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     return fp8 ? launch_decode<true, kStagesFp8>(prm, mk, mv, batch, num_kv_heads, st)
                : launch_decode<false, kStagesF16>(prm, mk, mv, batch, num_kv_heads, st);
+}
+
+pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
+                                 void* k_cache, void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_context_len,
+                                 float softmax_scale, int32_t kv_dtype, float k_scale, float v_scale,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                              num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                                              kv_dtype, k_scale, v_scale, PKV_PARTITION_AUTO);
+    if (v != PKV_OK || batch == 0) return v;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_INVALID_ARG;
+    if (!use_balanced(batch, num_kv_heads, max_blocks_per_seq)) return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+    if (grid <= 0) return PKV_ERR_CUDA;
+    return launch_balanced(fp8, grid, k_new, v_new, out, q, k_cache, v_cache, block_tables, context_lens,
+                           batch, num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks,
+                           max_context_len, softmax_scale, k_scale, v_scale, workspace, workspace_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

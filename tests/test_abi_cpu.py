@@ -76,6 +76,7 @@ def _attn(**kw):
     (dict(bs=32, mb=2), pkv.PKV_ERR_UNSUPPORTED),
     (dict(maxlen=65), pkv.PKV_ERR_INVALID_ARG),            # > max_blocks * bs
     (dict(P=20), pkv.PKV_ERR_INVALID_ARG),                 # not a multiple of bs
+    (dict(P=-2), pkv.PKV_ERR_INVALID_ARG),                 # below PKV_PARTITION_AUTO
     (dict(P=16), pkv.PKV_ERR_WORKSPACE),                   # split without workspace
     (dict(P=16, ws=A, wsb=64), pkv.PKV_ERR_WORKSPACE),     # too small
     (dict(dt=1, ks=0.0), pkv.PKV_ERR_INVALID_ARG),         # FP8 needs positive scales

@@ -106,7 +106,10 @@ def test_cache_write_flags_slot_outside_pool():
 
 
 # ------------------------------------------------------------- attention parity
-@pytest.mark.parametrize("P", [0, 16, 32])
+AUTO = pkv.PKV_PARTITION_AUTO
+
+
+@pytest.mark.parametrize("P", [0, 16, 32, AUTO])
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_tiny_config_f16(P, seed):
     r = _run(W.WORKLOADS["tiny"], seed)
@@ -123,7 +126,7 @@ REDUCED = {
 
 
 @pytest.mark.parametrize("name", sorted(REDUCED))
-@pytest.mark.parametrize("P", [0, 64, 512])
+@pytest.mark.parametrize("P", [0, 64, 512, AUTO])
 def test_reduced_configs(name, P):
     w = W.with_sizes(W.WORKLOADS[name], **REDUCED[name])
     for seed in (0, 3):
@@ -143,7 +146,7 @@ def test_full_size_configs_sampled(name):
                       + list(rng.choice(w.B, size=min(w.B, 6), replace=False))))
     ref = r.oracle(seqs=seqs)
     P_bench = w.partition_tokens or pkv.paged_gqa_decode_suggest_partition(w.B, w.Hkv, r.max_len)
-    for P in sorted({0, P_bench}):
+    for P in sorted({0, P_bench, AUTO}):
         out = host(r.attention(P))
         assert_attention_close(out[seqs], ref, f"{name} P={P}")
     assert pkv.pkv_device_error() == 0
@@ -164,6 +167,7 @@ def test_block_permutation_invariance_bitwise():
     w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=6, num_blocks=1024)
     r = _run(w, 4)
     out1 = host(r.attention(128))
+    auto1 = host(r.attention(AUTO))
     perm = np.random.default_rng(9).permutation(w.num_blocks)
     k2 = np.empty_like(r.k_host); v2 = np.empty_like(r.v_host)
     k2[perm] = r.k_host; v2[perm] = r.v_host
@@ -171,6 +175,8 @@ def test_block_permutation_invariance_bitwise():
     bt2 = np.where(bt >= 0, perm[np.maximum(bt, 0)], -1).astype(np.int32)
     out2 = host(r.attention(128, bt=dev(bt2), k=dev(k2), v=dev(v2)))
     assert np.array_equal(out1.view(np.uint16), out2.view(np.uint16))
+    auto2 = host(r.attention(AUTO, bt=dev(bt2), k=dev(k2), v=dev(v2)))
+    assert np.array_equal(auto1.view(np.uint16), auto2.view(np.uint16))
 
 
 def test_split_with_partition_covering_context_is_bitwise_single_pass():
@@ -186,18 +192,19 @@ def test_split_equals_single_within_tolerance_and_workspace_reuse():
     r = _run(w, 7)
     ref = r.oracle()
     B, Hq, D = r.q.shape
-    n = pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, 256)
-    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
-    outs = []
-    for _ in range(3):                                      # the same workspace, reused
-        out = torch.empty((B, Hq, D), dtype=torch.float16, device="cuda")
-        pkv.paged_gqa_decode_attention(out, r.q, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
-                                       softmax_scale=float(r.x["softmax_scale"]), partition_tokens=256,
-                                       workspace=ws)
-        outs.append(host(out))
-    for o in outs:
-        assert_attention_close(o, ref, "split 256")
-        assert np.array_equal(o.view(np.uint16), outs[0].view(np.uint16))
+    for P in (256, AUTO):
+        n = pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, P)
+        ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        outs = []
+        for _ in range(3):                                  # the same workspace, reused
+            out = torch.empty((B, Hq, D), dtype=torch.float16, device="cuda")
+            pkv.paged_gqa_decode_attention(out, r.q, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                                           softmax_scale=float(r.x["softmax_scale"]),
+                                           partition_tokens=P, workspace=ws)
+            outs.append(host(out))
+        for o in outs:
+            assert_attention_close(o, ref, f"split {P}")
+            assert np.array_equal(o.view(np.uint16), outs[0].view(np.uint16))
     assert_attention_close(host(r.attention(0)), ref, "single")
 
 
@@ -206,7 +213,7 @@ def test_poison_never_read_bitwise():
     xa = W.make_inputs(w, 8, poison=True)
     xb = W.make_inputs(w, 8, poison=False)
     ra, rb = DecodeRun(w, xa), DecodeRun(w, xb)
-    for P in (0, 64):
+    for P in (0, 64, AUTO):
         a, b = host(ra.attention(P)), host(rb.attention(P))
         assert np.isfinite(a.astype(np.float32)).all()
         assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
@@ -218,7 +225,7 @@ def test_fp8_poison_code_never_read():
     kq, vq = fp8_caches(x)                                  # NaN rows quantise to 0x7F
     assert (kq == 0x7F).any()
     r = DecodeRun(w, x, "fp8", kq, vq)
-    for P in (0, 32):
+    for P in (0, 32, AUTO):
         assert_attention_close(host(r.attention(P)), r.oracle(), f"fp8 poison P={P}")
 
 
@@ -227,9 +234,10 @@ def test_head_map_contiguous_groups():
     x = W.make_inputs(w, 10, poison=False)
     x["v_pool"][:] = np.arange(w.Hkv, dtype=np.float16)[None, None, :, None]
     r = DecodeRun(w, x)
-    out = host(r.attention(64)).astype(np.float64)
     expect = np.repeat(np.arange(w.Hkv, dtype=np.float64), w.group)[None, :, None]
-    assert np.array_equal(out, np.broadcast_to(expect, out.shape))
+    for P in (64, AUTO):
+        out = host(r.attention(P)).astype(np.float64)
+        assert np.array_equal(out, np.broadcast_to(expect, out.shape))
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (16, 4), (14, 2), (8, 1), (32, 4)])
@@ -237,14 +245,14 @@ def test_group_sizes(Hq, Hkv):
     w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=3, Hq=Hq, Hkv=Hkv, num_blocks=1024,
                      ctx=("uniform", 1, 1000))
     r = _run(w, 11)
-    for P in (0, 128):
+    for P in (0, 128, AUTO):
         assert_attention_close(host(r.attention(P)), r.oracle(), f"Hq={Hq} Hkv={Hkv} P={P}")
 
 
 def test_empty_contexts_give_zero_rows():
     w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=4, num_blocks=512, ctx=("fixed", (0, 33, 0, 700)))
     r = _run(w, 12)
-    for P in (0, 64):
+    for P in (0, 64, AUTO):
         out = host(r.attention(P))
         assert not out[0].any() and not out[2].any()
         assert_attention_close(out, r.oracle(), f"empty P={P}")
@@ -253,8 +261,9 @@ def test_empty_contexts_give_zero_rows():
 def test_all_contexts_empty_and_zero_max_len():
     w = W.with_sizes(W.WORKLOADS["tiny"], ctx=("fixed", (0, 0)))
     r = _run(w, 0)
-    out = host(r.attention(0, max_len=0))
-    assert not out.any()
+    for P in (0, AUTO):
+        out = host(r.attention(P, max_len=0))
+        assert not out.any()
 
 
 def test_bad_block_id_and_length_are_flagged_not_faulted():
@@ -277,7 +286,7 @@ def test_step_captured_in_cuda_graph():
     w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=8, num_blocks=2048)
     x = W.make_inputs(w, 13)
     r = DecodeRun(w, x)
-    P = 128
+    P = AUTO
     B, Hq, D = r.q.shape
     ws = torch.zeros(pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, P),
                      dtype=torch.uint8, device="cuda")
@@ -307,4 +316,136 @@ def test_step_captured_in_cuda_graph():
     ref = oracle.paged_gqa_decode(x["q"], kr, vr, x["block_tables"], x["context_lens"],
                                   float(x["softmax_scale"]))
     assert_attention_close(host(out), ref, "graph replay")
+    del g
+
+
+# ------------------------------------------------------- the balanced plan
+def test_auto_many_short_sequences():
+    """Thousands of 1..40-token sequences: many whole segments per worker."""
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=3000, num_blocks=9000, ctx=("uniform", 1, 40))
+    r = _run(w, 14)
+    seqs = np.random.default_rng(1).choice(w.B, 200, replace=False)
+    out = host(r.attention(AUTO))
+    assert_attention_close(out[np.sort(seqs)], r.oracle(seqs=np.sort(seqs)), "auto short")
+    assert pkv.pkv_device_error() == 0
+
+
+def test_auto_one_sequence_split_over_many_workers():
+    """One 32k-token sequence among short ones: its segments span hundreds of workers."""
+    w = W.with_sizes(W.WORKLOADS["skewed-split"], B=3, num_blocks=4096, ctx=("skewed", 32768, 2, 1, 50))
+    r = _run(w, 15)
+    assert_attention_close(host(r.attention(AUTO)), r.oracle(), "auto long")
+
+
+def test_auto_batch_beyond_balanced_tables_falls_back():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=9000, num_blocks=20000, ctx=("uniform", 1, 40))
+    r = _run(w, 16)
+    seqs = np.arange(0, w.B, 45)
+    out = host(r.attention(AUTO))
+    assert_attention_close(out[seqs], r.oracle(seqs=seqs), "auto fallback")
+
+
+# ------------------------------------------------------- fused decode step
+def _step(r, kn, vn, ws=None):
+    B, Hq, D = r.q.shape
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.float16, device="cuda")
+    if ws is None:
+        ws = torch.zeros(pkv.paged_gqa_decode_workspace_size(B, Hq, r.w.Hkv, D, r.max_len, AUTO),
+                         dtype=torch.uint8, device="cuda")
+    pkv.paged_gqa_decode_step(out, r.q, kn, vn, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                              softmax_scale=float(r.x["softmax_scale"]), kv_dtype=r.kv_dtype,
+                              k_scale=float(r.x["k_scale"]), v_scale=float(r.x["v_scale"]), workspace=ws)
+    torch.cuda.synchronize()
+    return out
+
+
+STEP_CASES = {
+    "tiny": {},
+    "qwen2.5-1.5b": dict(B=8),
+    "qwen2.5-7b": dict(B=6, num_blocks=2048),
+    "fp8-e4m3": dict(B=4, num_blocks=4096, ctx=("uniform", 1, 2600)),
+    "skewed-split": dict(B=4, num_blocks=1024, ctx=("skewed", 4100, 3, 1, 700)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(STEP_CASES))
+def test_fused_step_writes_cache_and_matches_oracle(name):
+    w = W.with_sizes(W.WORKLOADS[name], **STEP_CASES[name])
+    r = _run(w, 17)
+    x = r.x
+    out = host(_step(r, dev(x["k_new"]), dev(x["v_new"])))
+    kr, vr = r.k_host.copy(), r.v_host.copy()
+    oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"], kv_dtype=r.kv_dtype,
+                                k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    view = (lambda a: a.view(np.uint16)) if r.kv_dtype == "f16" else (lambda a: a)
+    assert np.array_equal(view(host(r.k)), view(kr))
+    assert np.array_equal(view(host(r.v)), view(vr))
+    ref = oracle.paged_gqa_decode(x["q"], kr, vr, x["block_tables"], x["context_lens"],
+                                  float(x["softmax_scale"]), kv_dtype=r.kv_dtype,
+                                  k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    assert_attention_close(out, ref, f"step {name}")
+    assert pkv.pkv_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["qwen2.5-1.5b", "fp8-e4m3"])
+def test_fused_step_equals_write_then_attention_bitwise(name):
+    w = W.with_sizes(W.WORKLOADS[name], **STEP_CASES[name])
+    x = W.make_inputs(w, 18)
+    if w.kv_dtype == "fp8":
+        kq, vq = fp8_caches(x)
+        r1, r2 = DecodeRun(w, x, "fp8", kq, vq), DecodeRun(w, x, "fp8", kq, vq)
+    else:
+        r1, r2 = DecodeRun(w, x), DecodeRun(w, x)
+    fused = host(_step(r1, dev(x["k_new"]), dev(x["v_new"])))
+    pkv.paged_kv_cache_write(dev(x["k_new"]), dev(x["v_new"]), r2.k, r2.v, dev(x["slot_mapping"]),
+                             kv_dtype=w.kv_dtype, k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    two = host(r2.attention(AUTO))
+    assert np.array_equal(fused.view(np.uint16), two.view(np.uint16))
+    bits = (lambda t: t.view(torch.int16)) if w.kv_dtype == "f16" else (lambda t: t)
+    assert torch.equal(bits(r1.k), bits(r2.k)) and torch.equal(bits(r1.v), bits(r2.v))
+
+
+@pytest.mark.parametrize("name", ["qwen2.5-1.5b", "qwen2.5-7b", "fp8-e4m3", "skewed-split"])
+def test_fused_step_full_size_sampled(name):
+    w = W.WORKLOADS[name]
+    r = _run(w, 19)
+    x = r.x
+    out = host(_step(r, dev(x["k_new"]), dev(x["v_new"])))
+    lens = x["context_lens"]
+    seqs = np.array(sorted(set([int(np.argmax(lens)), int(np.argmin(lens))]
+                               + list(np.random.default_rng(6).choice(w.B, min(w.B, 6), replace=False)))))
+    kr, vr = r.k_host, r.v_host                          # updated in place: only the new rows change
+    oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"], kv_dtype=r.kv_dtype,
+                                k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    ref = oracle.paged_gqa_decode(x["q"][seqs], kr, vr, x["block_tables"][seqs], lens[seqs],
+                                  float(x["softmax_scale"]), kv_dtype=r.kv_dtype,
+                                  k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    assert_attention_close(out[seqs], ref, f"step full {name}")
+    assert pkv.pkv_device_error() == 0
+
+
+def test_fused_step_empty_contexts_and_graph_replay():
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-7b"], B=5, num_blocks=1024, ctx=("fixed", (0, 33, 0, 700, 16)))
+    x = W.make_inputs(w, 20)
+    r = DecodeRun(w, x)
+    B, Hq, D = r.q.shape
+    ws = torch.zeros(pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, AUTO),
+                     dtype=torch.uint8, device="cuda")
+    kn, vn = dev(x["k_new"]), dev(x["v_new"])
+    _step(r, kn, vn, ws)                                   # warm-up outside the capture
+    g = torch.cuda.CUDAGraph()
+    out = torch.empty((B, Hq, D), dtype=torch.float16, device="cuda")
+    with torch.cuda.graph(g):
+        pkv.paged_gqa_decode_step(out, r.q, kn, vn, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                                  softmax_scale=float(x["softmax_scale"]), workspace=ws)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    kr, vr = x["k_pool"].copy(), x["v_pool"].copy()
+    oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"])
+    ref = oracle.paged_gqa_decode(x["q"], kr, vr, x["block_tables"], x["context_lens"],
+                                  float(x["softmax_scale"]))
+    o = host(out)
+    assert not o[0].any() and not o[2].any()
+    assert_attention_close(o, ref, "step graph")
     del g
