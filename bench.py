@@ -237,6 +237,8 @@ def parse_args(argv=None):
                     help="split-KV plan: -1 the library's balanced plan (default), 0 single pass, "
                          "P > 0 fixed partitions of P tokens")
     ap.add_argument("--graph-steps", type=int, default=500, help="steps per captured CUDA graph")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="fused step without PKV_STEP_OVERLAP_PREVIOUS")
     ap.add_argument("--unfused", action="store_true",
                     help="two launches per step (cache write, then attention) instead of the fused step")
     ap.add_argument("--no-e2e", action="store_true")
@@ -330,6 +332,7 @@ def run_ours(args):
     out = torch.empty((B, Hq, D), dtype=torch.float16, device=device)
 
     fused = not args.unfused and P == pkv.PKV_PARTITION_AUTO
+    step_flags = 0 if args.no_overlap else pkv.PKV_STEP_OVERLAP_PREVIOUS
 
     def cache_write(i):
         if fused:                                  # the step kernel writes the new tokens itself
@@ -341,9 +344,11 @@ def run_ours(args):
     def attention(i):
         kc, vc = pools[i % R]
         if fused:
+            # consecutive steps read different pool replicas, so no launch writes
+            # the pages the next one reads: the overlap promise holds
             pkv.paged_gqa_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, max_context_len=max_len,
                                       softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                      workspace=ws, stream=stream)
+                                      workspace=ws, flags=step_flags, stream=stream)
         else:
             pkv.paged_gqa_decode_attention(out, q, kc, vc, bt, cl, max_context_len=max_len,
                                            softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
@@ -360,16 +365,22 @@ def run_ours(args):
     S = max(1, min(args.graph_steps, K))
     chunks = [S] * (K // S) + ([K % S] if K % S else [])
     graphs, ev_pairs = {}, []
+    # Fused: one launch per step and nothing between launches, so that each
+    # launch overlaps the previous one's tail (programmatic dependent launch);
+    # its average duration is the timed region over K. Unfused: events around
+    # every attention launch give that kernel's own duration.
     for n in sorted(set(chunks)):
-        evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
+        evs = [] if fused else [(torch.cuda.Event(enable_timing=True, external=True),
+                                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
                 cache_write(i)
-                evs[i][0].record(stream)
+                if evs:
+                    evs[i][0].record(stream)
                 attention(i)
-                evs[i][1].record(stream)
+                if evs:
+                    evs[i][1].record(stream)
         graphs[n] = (g, evs)
     torch.cuda.synchronize()
 
@@ -387,10 +398,12 @@ def run_ours(args):
     wall1 = time.perf_counter()
     barrier(world, device)
     sampler.stop()
-    # per-launch durations of the attention kernel in the last replay of each graph
-    for n in set(chunks):
-        attn_ms += [a.elapsed_time(b) for a, b in graphs[n][1]]
     elapsed_ms = start.elapsed_time(end)
+    if fused:
+        attn_ms = [elapsed_ms / K]
+    else:        # per-launch durations of the attention kernel in the last replay of each graph
+        for n in set(chunks):
+            attn_ms += [a.elapsed_time(b) for a, b in graphs[n][1]]
     elapsed_max = reduce_max(elapsed_ms, world, device)
     launches = (1 if fused else 2) * K
 
@@ -459,8 +472,9 @@ def run_ours(args):
                        "l2": f"inputs larger than L2: {R} KV pool replicas rotated, "
                              f"{R * touched / 2**20:.0f} MiB touched per cycle",
                        "timing": f"{len(chunks)} CUDA graph replays of <= {S} steps",
-                       "step": "one fused launch (cache write + attention)" if fused
-                               else "cache write + attention launches"},
+                       "step": ("one fused launch (cache write + attention)" +
+                                ("" if args.no_overlap else ", PKV_STEP_OVERLAP_PREVIOUS"))
+                               if fused else "cache write + attention launches"},
             "roofline": {"bound": "hbm",
                          "kernel": "decode_balanced_kernel (fused step)" if fused else "decode attention",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",

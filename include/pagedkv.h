@@ -86,6 +86,9 @@ typedef enum {
  * equal share of the batch's pages, whatever the length mix). */
 #define PKV_PARTITION_AUTO (-1)
 
+/* flags of paged_gqa_decode_step */
+#define PKV_STEP_OVERLAP_PREVIOUS 0x1u
+
 /* Bits of the device error word (pkv_device_error). */
 #define PKV_DEVERR_CONTEXT_LEN   0x1u  /* a context length exceeded max_context_len or the
                                           table capacity; it was clamped */
@@ -200,7 +203,20 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q,
  * row in shared memory and writes it to the cache, so no second launch is
  * needed. Always the load-balanced plan: `workspace` as for
  * paged_gqa_decode_attention with PKV_PARTITION_AUTO (zero-filled before its
- * first use). Batches above 8192 sequences return PKV_ERR_UNSUPPORTED.
+ * first use). Batches whose tables do not fit the kernel's shared memory
+ * (above 8192 sequences) return PKV_ERR_UNSUPPORTED.
+ *
+ * flags: 0, or PKV_STEP_OVERLAP_PREVIOUS. The kernel is launched with
+ * programmatic dependent launch, so it may start while the previous launch
+ * in `stream` finishes. By default it waits for that launch before reading
+ * any input. With PKV_STEP_OVERLAP_PREVIOUS it first reads context_lens,
+ * block_tables and the cache pages and only then waits (before q, k_new,
+ * v_new, the workspace and out): the caller promises that the launch
+ * immediately before this one in `stream` writes none of context_lens,
+ * block_tables and the cache pages. In a layer loop, where the step follows
+ * the QKV projection and the pages were written by earlier steps, this lets
+ * the first page loads overlap the previous kernel. A prefill or a separate
+ * cache write launched just before the step breaks the promise.
  */
 pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
                                  void* k_cache, void* v_cache,
@@ -210,7 +226,8 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
                                  int32_t max_blocks_per_seq, int32_t num_blocks,
                                  int32_t max_context_len, float softmax_scale,
                                  int32_t kv_dtype, float k_scale, float v_scale,
-                                 void* workspace, size_t workspace_bytes, void* stream);
+                                 void* workspace, size_t workspace_bytes, uint32_t flags,
+                                 void* stream);
 
 /* Static text for a status code. Never NULL. */
 const char* pkv_status_string(pkv_status status);

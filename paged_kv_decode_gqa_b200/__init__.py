@@ -32,7 +32,7 @@ _SIGNATURES = {
     "paged_gqa_decode_attention": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                     _i32, _f32, _i32, _f32, _f32, _i32, _P, _sz, _P], ctypes.c_int),
     "paged_gqa_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
-                               _i32, _f32, _i32, _f32, _f32, _P, _sz, _P], ctypes.c_int),
+                               _i32, _f32, _i32, _f32, _f32, _P, _sz, ctypes.c_uint32, _P], ctypes.c_int),
     "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "pkv_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
     "paged_gqa_decode_attention_static_workspace": (
@@ -71,6 +71,7 @@ def __getattr__(name):
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_WORKSPACE, PKV_ERR_CUDA = range(5)
 PKV_KV_F16, PKV_KV_FP8_E4M3 = 0, 1
 PKV_PARTITION_AUTO = -1         # partition_tokens: the library's load-balanced plan
+PKV_STEP_OVERLAP_PREVIOUS = 0x1  # paged_gqa_decode_step flag (see include/pagedkv.h)
 DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 _KV_DTYPES = {"f16": PKV_KV_F16, "fp8": PKV_KV_FP8_E4M3}
 
@@ -171,7 +172,7 @@ def paged_gqa_decode_attention(out, q, k_cache, v_cache, block_tables, context_l
 
 def paged_gqa_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, *,
                           max_context_len, softmax_scale, kv_dtype="f16", k_scale=1.0, v_scale=1.0,
-                          workspace=None, stream=None) -> None:
+                          workspace=None, flags=0, stream=None) -> None:
     """One decode step in one launch: k_new/v_new [B, Hkv, D] go to position
     context_lens[b] - 1 of each sequence's pages, then out = attention over the
     updated cache (the load-balanced plan; workspace sized for PKV_PARTITION_AUTO)."""
@@ -193,7 +194,7 @@ def paged_gqa_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, 
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
         float(softmax_scale), kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _ptr(workspace),
-        ws_bytes, _stream(stream)), "paged_gqa_decode_step")
+        ws_bytes, int(flags), _stream(stream)), "paged_gqa_decode_step")
 
 
 def pkv_device_error() -> int:

@@ -48,6 +48,7 @@ struct BalancedParams {
     int32_t B, Hq, Hkv, G;
     int32_t max_blocks_per_seq, num_blocks, max_context_len;
     int32_t min_units_per_worker;
+    int32_t overlap_previous;     // read pages/tables/lengths before waiting on the previous launch
     float logit_scale_log2;       // softmax_scale * log2(e) (* k_scale for FP8)
     float out_scale;              // 1 (v_scale for FP8)
 };
@@ -120,9 +121,11 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     const uint32_t bars = ring + S::kRingBytes + (uint32_t)(((2 * B + 1) * 4 + 15) / 16 * 16) +
                           (uint32_t)(kWarps * kMergeFloats * 4);
 
-    // Everything above touched only shared memory; inputs may come from the
-    // previous launch in the stream.
-    grid_dependency_wait();
+    // Everything above touched only shared memory. Inputs may come from the
+    // previous launch in the stream: wait for it here, unless the caller
+    // declared that it writes none of the KV pages, tables and lengths read
+    // before the second wait point below (overlap_previous).
+    if (!p.overlap_previous) grid_dependency_wait();
     grid_dependents_launch();
 
     // ---- unit order: units of sequence b start at prefix[b] ----
@@ -161,24 +164,27 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         mbar_init_fence();
         __syncthreads();
     }
-    // empty contexts: zero rows, spread over the CTAs
-    for (int b = blockIdx.x; b < B; b += gridDim.x) {
-        if (lens[b] != 0) continue;
-        __half* ob = p.out + (int64_t)b * p.Hq * kHeadDim;
-        for (int i = threadIdx.x; i < p.Hq * kHeadDim; i += S::kThreads) ob[i] = __float2half_rn(0.f);
-    }
-
     // ---- this warp's range of units ----
     const int U = prefix[B];
     const int W_total = gridDim.x * kWarps;
-    if (U == 0) return;
+    const int worker = blockIdx.x * kWarps + warp;
+    // empty contexts get zero rows, spread over all warps (after the wait)
+    auto zero_rows = [&]() {
+        for (int bb = worker; bb < B; bb += W_total) {
+            if (lens[bb] != 0) continue;
+            uint4* ob = reinterpret_cast<uint4*>(p.out + (int64_t)bb * p.Hq * kHeadDim);
+            for (int i = lane; i < p.Hq * kHeadDim / 8; i += 32) ob[i] = make_uint4(0, 0, 0, 0);
+        }
+    };
     const int want = (U + p.min_units_per_worker - 1) / p.min_units_per_worker;
     const int W = min(W_total, max(1, want));
-    const int worker = blockIdx.x * kWarps + warp;
-    if (worker >= W) return;
-    const int u0 = (int)range_start(worker, U, W);
-    const int n = (int)range_start(worker + 1, U, W) - u0;
-    if (n <= 0) return;
+    const int u0 = U == 0 ? 0 : (int)range_start(worker, U, W);
+    const int n = (U == 0 || worker >= W) ? 0 : (int)range_start(worker + 1, U, W) - u0;
+    if (n <= 0) {
+        if (p.overlap_previous) grid_dependency_wait();
+        zero_rows();
+        return;
+    }
     if (lane == 0) {
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
@@ -241,6 +247,9 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     };
     const int prologue = min(n, kStages);
     for (int t = 0; t < prologue; ++t) issue(t);
+    // From here on: q, this step's new tokens, the workspace and out, which
+    // the previous launch may produce or still use.
+    if (p.overlap_previous) grid_dependency_wait();
 
     // ---- stream the range ----
     const int r = lane >> 2, c = lane & 3;
@@ -317,28 +326,37 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int first = item & ~31, last = min(first + 32, n_items) - 1;
             const int cslot = slot_of_piece(first * span);
             unsigned int* cnt = p.ws_count + (int64_t)lvl * 2 * W_total + cslot;
-            // the warp barrier orders every lane's stores before lane 0's fence
+            // The warp barrier orders every lane's stores before lane 0's
+            // release-acquire ticket; the merger's loads follow its acquire.
             __syncwarp();
             unsigned int prev = 0;
-            if (lane == 0) {
-                __threadfence();
-                prev = atomicAdd(cnt, 1u);
-                __threadfence();
-            }
+            if (lane == 0) prev = atomic_add_acq_rel_gpu(cnt, 1u);
             prev = __shfl_sync(0xffffffffu, prev, 0);
             if (prev != (unsigned int)(last - first)) return;   // another item merges the group
-            // ---- merge items first..last: weights lane-parallel, values unrolled ----
+            // ---- merge items first..last ----
+            // (m, l) lane-parallel and the first two items' values are loaded
+            // together; later values are double-buffered two items at a time.
             const int n_it = last - first + 1;
             const int my_slot = lane < n_it ? slot_of_piece((first + lane) * span) : 0;
-            float mm[8], ll[8];
-            {
-                const int sl = my_slot;
+            auto load_vals = [&](float4 (&dst)[2][8], int t) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float4 a = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-                    if (lane < n_it) a = __ldcg(p.ws_ml + (int64_t)sl * 4 + k);
-                    mm[2 * k] = a.x; ll[2 * k] = a.y; mm[2 * k + 1] = a.z; ll[2 * k + 1] = a.w;
+                for (int u = 0; u < 2; ++u) {
+                    if (t + u < n_it) {
+                        const int sl = __shfl_sync(0xffffffffu, my_slot, t + u);
+                        const float4* src = p.ws_o + ((int64_t)sl * 32 + lane) * 8;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) dst[u][i] = __ldcg(src + i);
+                    }
                 }
+            };
+            float4 va[2][8], vb[2][8];
+            load_vals(va, 0);
+            float mm[8], ll[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float4 a = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+                if (lane < n_it) a = __ldcg(p.ws_ml + (int64_t)my_slot * 4 + k);
+                mm[2 * k] = a.x; ll[2 * k] = a.y; mm[2 * k + 1] = a.z; ll[2 * k + 1] = a.w;
             }
 #pragma unroll
             for (int h = 0; h < 8; ++h) {
@@ -359,28 +377,24 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             float acc[8][4];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-            for (int t0 = 0; t0 < n_it; t0 += 4) {
-                float4 val[4][8];
+            auto consume = [&](const float4 (&vals)[2][8], int t) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (t0 + u < n_it) {
-                        const int sl = __shfl_sync(0xffffffffu, my_slot, t0 + u);
-                        const float4* src = p.ws_o + ((int64_t)sl * 32 + lane) * 8;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) val[u][i] = __ldcg(src + i);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (t0 + u < n_it) {
-                        const float w0 = wts[(t0 + u) * 8 + 2 * c], w1 = wts[(t0 + u) * 8 + 2 * c + 1];
+                for (int u = 0; u < 2; ++u) {
+                    if (t + u < n_it) {
+                        const float w0 = wts[(t + u) * 8 + 2 * c], w1 = wts[(t + u) * 8 + 2 * c + 1];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            acc[i][0] += w0 * val[u][i].x; acc[i][1] += w1 * val[u][i].y;
-                            acc[i][2] += w0 * val[u][i].z; acc[i][3] += w1 * val[u][i].w;
+                            acc[i][0] += w0 * vals[u][i].x; acc[i][1] += w1 * vals[u][i].y;
+                            acc[i][2] += w0 * vals[u][i].z; acc[i][3] += w1 * vals[u][i].w;
                         }
                     }
                 }
+            };
+            for (int t0 = 0; t0 < n_it; t0 += 4) {
+                if (t0 + 2 < n_it) load_vals(vb, t0 + 2);
+                consume(va, t0);
+                if (t0 + 4 < n_it) load_vals(va, t0 + 4);
+                if (t0 + 2 < n_it) consume(vb, t0 + 2);
             }
             m0 = wts[256 + 2 * c]; m1 = wts[256 + 2 * c + 1];
             l0 = wts[264 + 2 * c]; l1 = wts[264 + 2 * c + 1];
@@ -471,6 +485,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             ++j;
         }
     }
+    zero_rows();
 }
 
 }  // namespace pkv

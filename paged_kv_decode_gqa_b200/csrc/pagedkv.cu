@@ -26,11 +26,21 @@ constexpr int kConsumers = 4;
 constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
 constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 
-// Balanced streaming kernel: 4 worker warps per CTA, each with its own ring
-// of page slots (f16: 3 x 8 KiB, FP8: 6 x 4 KiB), two CTAs per SM.
-constexpr int kBalWarps = 4;
-constexpr int kBalStagesF16 = 3;
-constexpr int kBalStagesFp8 = 6;
+// Balanced streaming kernel: worker warps per CTA and page slots per worker
+// ring (f16 pages are 8 KiB, FP8 pages 4 KiB). The defaults give 96 KiB of
+// ring per CTA and two CTAs per SM; the macros exist for tuning builds.
+#ifndef PKV_BAL_WARPS
+#define PKV_BAL_WARPS 4
+#endif
+#ifndef PKV_BAL_STAGES_F16
+#define PKV_BAL_STAGES_F16 3
+#endif
+#ifndef PKV_BAL_STAGES_FP8
+#define PKV_BAL_STAGES_FP8 6
+#endif
+constexpr int kBalWarps = PKV_BAL_WARPS;
+constexpr int kBalStagesF16 = PKV_BAL_STAGES_F16;
+constexpr int kBalStagesFp8 = PKV_BAL_STAGES_FP8;
 constexpr int kBalMaxBatch = 8192;        // unit-order tables must fit in shared memory
 constexpr int kBalMinUnits = 4;           // pages per worker at least (small batches)
 
@@ -159,14 +169,17 @@ template <bool kFp8>
 int balanced_grid(int B) {
     static unsigned long long done = 0, done_fused = 0;
     auto kernel = balanced_kernel<kFp8>();
-    if (ensure_smem(balanced_kernel<kFp8, true>(), (int)BalShape<kFp8>::smem_bytes(kBalMaxBatch),
-                    &done_fused) != cudaSuccess)
-        return 0;
-    if (ensure_smem(kernel, (int)BalShape<kFp8>::smem_bytes(kBalMaxBatch), &done) != cudaSuccess) return 0;
-    int dev = 0, sms = 0, per_sm = 0;
+    int dev = 0, sms = 0, per_sm = 0, optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return 0;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return 0;
+    const int dyn_max = optin - (int)fa.sharedSizeBytes;            // opt-in minus static shared
+    if (BalShape<kFp8>::smem_bytes(B) > (size_t)dyn_max) return 0;  // tables do not fit
+    if (ensure_smem(balanced_kernel<kFp8, true>(), dyn_max, &done_fused) != cudaSuccess) return 0;
+    if (ensure_smem(kernel, dyn_max, &done) != cudaSuccess) return 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, BalShape<kFp8>::kThreads,
                                                       BalShape<kFp8>::smem_bytes(B)) != cudaSuccess)
         return 0;
@@ -204,7 +217,8 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
                            const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
                            int32_t Hq, int32_t Hkv, int32_t max_blocks_per_seq, int32_t num_blocks,
                            int32_t max_context_len, float softmax_scale, float k_scale, float v_scale,
-                           void* workspace, size_t workspace_bytes, cudaStream_t st) {
+                           void* workspace, size_t workspace_bytes, bool overlap_previous,
+                           cudaStream_t st) {
     const BalancedLayout bl = balanced_layout((int64_t)grid * kBalWarps, batch, Hkv);
     if (!workspace || workspace_bytes < bl.total) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
@@ -231,6 +245,7 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
     bp.num_blocks = num_blocks;
     bp.max_context_len = max_context_len;
     bp.min_units_per_worker = kBalMinUnits;
+    bp.overlap_previous = overlap_previous ? 1 : 0;
     const float log2e = 1.4426950408889634f;
     bp.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
     bp.out_scale = fp8 ? v_scale : 1.f;
@@ -363,11 +378,9 @@ size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
         return 0;
     if (partition_tokens == PKV_PARTITION_AUTO) {
         const int64_t max_blocks = std::max(1, (max_context_len + kPageRows - 1) / kPageRows);
-        if (use_balanced(batch, num_kv_heads, max_blocks)) {
-            const int grid = std::max(balanced_grid<false>(batch), balanced_grid<true>(batch));
-            if (grid <= 0) return 0;
-            return balanced_layout((int64_t)grid * kBalWarps, batch, num_kv_heads).total;
-        }
+        const int grid = use_balanced(batch, num_kv_heads, max_blocks)
+                             ? std::max(balanced_grid<false>(batch), balanced_grid<true>(batch)) : 0;
+        if (grid > 0) return balanced_layout((int64_t)grid * kBalWarps, batch, num_kv_heads).total;
         partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
                                                               kPageRows, 0);
     }
@@ -419,13 +432,13 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
     const float log2e = 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (partition_tokens == PKV_PARTITION_AUTO) {
-        if (use_balanced(batch, num_kv_heads, max_blocks_per_seq)) {
-            const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
-            if (grid <= 0) return PKV_ERR_CUDA;
+        const int grid = !use_balanced(batch, num_kv_heads, max_blocks_per_seq) ? 0
+                         : fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+        if (grid > 0) {
             return launch_balanced(fp8, grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
                                    context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
                                    num_blocks, max_context_len, softmax_scale, k_scale, v_scale,
-                                   workspace, workspace_bytes, st);
+                                   workspace, workspace_bytes, false, st);
         }
         partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
                                                               kPageRows, 0);
@@ -477,7 +490,8 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
                                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                  int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_context_len,
                                  float softmax_scale, int32_t kv_dtype, float k_scale, float v_scale,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+                                 void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
+    if (flags & ~PKV_STEP_OVERLAP_PREVIOUS) return PKV_ERR_INVALID_ARG;
     const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                               num_q_heads, num_kv_heads, head_dim, block_size,
                                               max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
@@ -487,11 +501,11 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
     if (!use_balanced(batch, num_kv_heads, max_blocks_per_seq)) return PKV_ERR_UNSUPPORTED;
     const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
     const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
-    if (grid <= 0) return PKV_ERR_CUDA;
+    if (grid <= 0) return PKV_ERR_UNSUPPORTED;
     return launch_balanced(fp8, grid, k_new, v_new, out, q, k_cache, v_cache, block_tables, context_lens,
                            batch, num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks,
                            max_context_len, softmax_scale, k_scale, v_scale, workspace, workspace_bytes,
-                           static_cast<cudaStream_t>(stream));
+                           (flags & PKV_STEP_OVERLAP_PREVIOUS) != 0, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

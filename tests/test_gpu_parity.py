@@ -346,7 +346,7 @@ def test_auto_batch_beyond_balanced_tables_falls_back():
 
 
 # ------------------------------------------------------- fused decode step
-def _step(r, kn, vn, ws=None):
+def _step(r, kn, vn, ws=None, flags=0):
     B, Hq, D = r.q.shape
     out = torch.full((B, Hq, D), float("nan"), dtype=torch.float16, device="cuda")
     if ws is None:
@@ -354,7 +354,8 @@ def _step(r, kn, vn, ws=None):
                          dtype=torch.uint8, device="cuda")
     pkv.paged_gqa_decode_step(out, r.q, kn, vn, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
                               softmax_scale=float(r.x["softmax_scale"]), kv_dtype=r.kv_dtype,
-                              k_scale=float(r.x["k_scale"]), v_scale=float(r.x["v_scale"]), workspace=ws)
+                              k_scale=float(r.x["k_scale"]), v_scale=float(r.x["v_scale"]), workspace=ws,
+                              flags=flags)
     torch.cuda.synchronize()
     return out
 
@@ -368,12 +369,13 @@ STEP_CASES = {
 }
 
 
+@pytest.mark.parametrize("flags", [0, pkv.PKV_STEP_OVERLAP_PREVIOUS])
 @pytest.mark.parametrize("name", sorted(STEP_CASES))
-def test_fused_step_writes_cache_and_matches_oracle(name):
+def test_fused_step_writes_cache_and_matches_oracle(name, flags):
     w = W.with_sizes(W.WORKLOADS[name], **STEP_CASES[name])
     r = _run(w, 17)
     x = r.x
-    out = host(_step(r, dev(x["k_new"]), dev(x["v_new"])))
+    out = host(_step(r, dev(x["k_new"]), dev(x["v_new"]), flags=flags))
     kr, vr = r.k_host.copy(), r.v_host.copy()
     oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"], kv_dtype=r.kv_dtype,
                                 k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
@@ -448,4 +450,42 @@ def test_fused_step_empty_contexts_and_graph_replay():
     o = host(out)
     assert not o[0].any() and not o[2].any()
     assert_attention_close(o, ref, "step graph")
+    del g
+
+
+def test_fused_steps_back_to_back_with_overlap_flag():
+    """Steps on alternating pools with PKV_STEP_OVERLAP_PREVIOUS, in a graph: each
+    step's output matches the oracle (the promise holds: consecutive steps use
+    different pools and tables)."""
+    w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=16, num_blocks=2048)
+    xs = [W.make_inputs(w, 30 + i) for i in range(2)]
+    rs = [DecodeRun(w, x) for x in xs]
+    B, Hq, D = rs[0].q.shape
+    ws = torch.zeros(pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, 2048, AUTO),
+                     dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((B, Hq, D), dtype=torch.float16, device="cuda") for _ in range(2)]
+    kns = [(dev(x["k_new"]), dev(x["v_new"])) for x in xs]
+
+    def steps():
+        for i in range(6):
+            r, (kn, vn) = rs[i % 2], kns[i % 2]
+            pkv.paged_gqa_decode_step(outs[i % 2], r.q, kn, vn, r.k, r.v, r.bt, r.cl, max_context_len=2048,
+                                      softmax_scale=float(r.x["softmax_scale"]), workspace=ws,
+                                      flags=pkv.PKV_STEP_OVERLAP_PREVIOUS)
+
+    steps()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        steps()
+    for o in outs:
+        o.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    for i, (x, o) in enumerate(zip(xs, outs)):
+        kr, vr = x["k_pool"].copy(), x["v_pool"].copy()
+        oracle.paged_kv_cache_write(x["k_new"], x["v_new"], kr, vr, x["slot_mapping"])
+        ref = oracle.paged_gqa_decode(x["q"], kr, vr, x["block_tables"], x["context_lens"],
+                                      float(x["softmax_scale"]))
+        assert_attention_close(host(o), ref, f"overlapped steps, pool {i}")
     del g
