@@ -21,7 +21,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIBRARY_PATH = os.path.join(_HERE, "libpagedkv_b200.so")
+# PKV_LIBRARY may name another build of the same library (e.g. a tuning build).
+LIBRARY_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpagedkv_b200.so")
 
 _P, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 _SIGNATURES = {

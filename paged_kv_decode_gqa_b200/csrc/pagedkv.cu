@@ -27,10 +27,12 @@ constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
 constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 
 // Balanced streaming kernel: worker warps per CTA and page slots per worker
-// ring (f16 pages are 8 KiB, FP8 pages 4 KiB). The defaults give 96 KiB of
-// ring per CTA and two CTAs per SM; the macros exist for tuning builds.
+// ring (f16 pages are 8 KiB, FP8 pages 4 KiB). The defaults -- 8 workers with
+// 3 f16 (6 FP8) slots each, 192 KiB of ring, one CTA per SM -- measured best
+// or near best on every benchmark workload among 4x3 (two CTAs per SM), 4x6,
+// 6x4 and 8x3; the macros exist for tuning builds.
 #ifndef PKV_BAL_WARPS
-#define PKV_BAL_WARPS 4
+#define PKV_BAL_WARPS 8
 #endif
 #ifndef PKV_BAL_STAGES_F16
 #define PKV_BAL_STAGES_F16 3
