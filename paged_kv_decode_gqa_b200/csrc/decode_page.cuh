@@ -76,7 +76,9 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
     const int r = lane >> 2, c = lane & 3;
 
     // ---- S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T ----
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    // Two independent accumulators (even and odd k-steps) halve the chain of
+    // dependent tensor-core ops; their sum is the contraction over all channels.
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     {
         const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
         if constexpr (!kFp8) {
@@ -86,7 +88,7 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
                 const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
                 uint32_t a0, a1, a2, a3;
                 ldsm_x4(addr, a0, a1, a2, a3);
-                mma_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                mma_16816(sacc[kk & 1], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
             }
         } else {
 #pragma unroll
@@ -95,10 +97,10 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
                 const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
                 uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
                 ldsm_x4(addr, r0, r1, r2, r3);
-                mma_16816(sacc, e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
+                mma_16816(sacc[0], e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
                           e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
                           qf[2 * J][0], qf[2 * J][1]);
-                mma_16816(sacc, e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
+                mma_16816(sacc[1], e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
                           e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
                           qf[2 * J + 1][0], qf[2 * J + 1][1]);
             }
@@ -106,7 +108,8 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
     }
 
     // ---- online softmax over this page's tokens (rows r, r+8) ----
-    float x0 = sacc[0] * sl, x1 = sacc[1] * sl, x2 = sacc[2] * sl, x3 = sacc[3] * sl;
+    float x0 = (sacc[0][0] + sacc[1][0]) * sl, x1 = (sacc[0][1] + sacc[1][1]) * sl;
+    float x2 = (sacc[0][2] + sacc[1][2]) * sl, x3 = (sacc[0][3] + sacc[1][3]) * sl;
     if (valid < kPageRows) {                    // rows past the context: excluded
         if (r >= valid) x0 = x1 = -INFINITY;
         if (r + 8 >= valid) x2 = x3 = -INFINITY;

@@ -330,6 +330,19 @@ def test_auto_many_short_sequences():
     assert pkv.pkv_device_error() == 0
 
 
+@pytest.mark.parametrize("kv_dtype", ["f16", "fp8"])
+def test_auto_many_segments_per_cta(kv_dtype):
+    """1500 sequences of 1..100 tokens: a few dozen segments per SM's range, most of them
+    split over several consumer warps, so the per-CTA accumulators are reused many times."""
+    base = W.WORKLOADS["fp8-e4m3" if kv_dtype == "fp8" else "qwen2.5-1.5b"]
+    w = W.with_sizes(base, B=1500, num_blocks=12000, ctx=("uniform", 1, 100))
+    r = _run(w, 17)
+    seqs = np.sort(np.random.default_rng(2).choice(w.B, 150, replace=False))
+    out = host(r.attention(AUTO))
+    assert_attention_close(out[seqs], r.oracle(seqs=seqs), f"auto many segments {kv_dtype}")
+    assert pkv.pkv_device_error() == 0
+
+
 def test_auto_one_sequence_split_over_many_workers():
     """One 32k-token sequence among short ones: its segments span hundreds of workers."""
     w = W.with_sizes(W.WORKLOADS["skewed-split"], B=3, num_blocks=4096, ctx=("skewed", 32768, 2, 1, 50))
