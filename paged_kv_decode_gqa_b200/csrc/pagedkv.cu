@@ -66,6 +66,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // View of one cache tensor [num_blocks, 16, Hkv, 128] as a 3-D TMA tensor
 // (channel, head, pool row) with 16-row x 128-byte boxes, 128-byte swizzled.
+// L2 fills are promoted to one KV head's row: 256 bytes in f16 (both boxes of
+// the row), 128 bytes in FP8, where a wider fill would drag in the next KV
+// head's row, which is streamed by another worker much later.
 bool make_cache_map(CUtensorMap* map, const void* base, bool fp8, int num_blocks, int Hkv) {
     PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
     if (!encode) return false;
@@ -77,7 +80,8 @@ bool make_cache_map(CUtensorMap* map, const void* base, bool fp8, int num_blocks
     CUresult r = encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                         const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        fp8 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
