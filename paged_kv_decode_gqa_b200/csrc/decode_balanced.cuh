@@ -101,11 +101,23 @@ __device__ __forceinline__ uint32_t quantize4_e4m3(uint2 x, float scale) {
     return out;
 }
 
+// Two consecutive pages of one segment per online-softmax step (when the
+// segment has them in the worker's range): two independent logit chains and
+// one max / rescale / shuffle round per 32 tokens. Measured faster for both
+// cache types (FP8 0.69 -> 0.78, Qwen2.5-7B f16 0.84 -> 0.91 of the copy peak).
+#ifndef PKV_PAGE_PAIRS_FP8
+#define PKV_PAGE_PAIRS_FP8 1
+#endif
+#ifndef PKV_PAGE_PAIRS_F16
+#define PKV_PAGE_PAIRS_F16 1
+#endif
+
 template <bool kFp8, int kWarps, int kStages, bool kFuseWrite>
 __global__ void __launch_bounds__(32 * kWarps)
 decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const BalancedParams p) {
     using S = BalancedShape<kFp8, kWarps, kStages>;
+    constexpr bool kPagePairs = (kFp8 ? PKV_PAGE_PAIRS_FP8 : PKV_PAGE_PAIRS_F16) && kStages >= 2;
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_warp_sum[kWarps];
 
@@ -421,12 +433,12 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     // in the cache for later ones. Lane l holds channels 4l..4l+3. The page's
     // TMA copy may hold the row's old contents; the shared row is overwritten
     // after the copy landed, so attention sees the new token either way.
-    auto write_new_token = [&](int s) {
+    auto write_new_token = [&](int s, int jl) {          // jl = nb - 1, the segment's last page
         const int row = (lens[b] - 1) & (kPageRows - 1);
         const int64_t src = ((int64_t)b * Hkv + g) * kHeadDim + 4 * lane;
         const uint2 kh = __ldg(reinterpret_cast<const uint2*>(p.k_new + src));
         const uint2 vh = __ldg(reinterpret_cast<const uint2*>(p.v_new + src));
-        const int pb = __ldg(p.block_tables + (int64_t)b * p.max_blocks_per_seq + j);
+        const int pb = __ldg(p.block_tables + (int64_t)b * p.max_blocks_per_seq + jl);
         const bool in_pool = pb >= 0 && pb < p.num_blocks;
         const int64_t dst = (((int64_t)pb * kPageRows + row) * Hkv + g) * kHeadDim + 4 * lane;
         if constexpr (kFp8) {
@@ -457,13 +469,29 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     for (int t = 0; t < n; ++t) {
         const int s = t % kStages;
         if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (t / kStages) & 1))) return;
-        const int valid = j == nb - 1 ? lens[b] - j * kPageRows : kPageRows;
-        if constexpr (kFuseWrite) {
-            if (j == nb - 1) write_new_token(s);    // this page holds position L - 1
+        if (kPagePairs && j + 1 < nb && t + 1 < n) {
+            // pages t and t + 1 are consecutive pages of one segment: one softmax step
+            const int s2 = (t + 1) % kStages;
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s2), ((t + 1) / kStages) & 1))) return;
+            const int valid_b = j + 1 == nb - 1 ? lens[b] - (j + 1) * kPageRows : kPageRows;
+            if constexpr (kFuseWrite) {
+                if (j + 1 == nb - 1) write_new_token(s2, j + 1);   // page B holds position L - 1
+            }
+            attend_page_pair<kFp8>(st, k_tile(s), v_tile(s), k_tile(s2), v_tile(s2), valid_b, qf, sl, lane);
+            __syncwarp();
+            if (t + kStages < n) issue(t + kStages);
+            if (t + 1 + kStages < n) issue(t + 1 + kStages);
+            ++t;                                   // the cursor moves to page B
+            ++j;
+        } else {
+            const int valid = j == nb - 1 ? lens[b] - j * kPageRows : kPageRows;
+            if constexpr (kFuseWrite) {
+                if (j == nb - 1) write_new_token(s, j);    // this page holds position L - 1
+            }
+            attend_page<kFp8>(st, k_tile(s), v_tile(s), valid, qf, sl, lane);
+            __syncwarp();
+            if (t + kStages < n) issue(t + kStages);
         }
-        attend_page<kFp8>(st, k_tile(s), v_tile(s), valid, qf, sl, lane);
-        __syncwarp();
-        if (t + kStages < n) issue(t + kStages);
         // advance the cursor; a segment boundary (or the range end) closes the piece
         const bool seg_end = j == nb - 1;
         if (seg_end || t == n - 1) {

@@ -67,76 +67,57 @@ __device__ __forceinline__ void load_q_fragments(uint32_t (&qf)[8][2], const __h
     }
 }
 
-// Online-softmax update of `st` with one page: K tile at shared address kt, V
-// tile at vt (f16: two 2 KiB boxes of 64 channels each; FP8: one 2 KiB box),
-// the first `valid` rows live. `sl` = softmax scale * log2(e) (* k_scale).
+// Logits S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T of one page, times
+// `sl`, with the rows at or past `valid` set to -inf: lane (r, c) gets tokens
+// r (x[0], x[1]) and r + 8 (x[2], x[3]) of heads 2c, 2c + 1. K tile at shared
+// address kt (f16: two 2 KiB boxes of 64 channels each; FP8: one 2 KiB box).
 template <bool kFp8>
-__device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t vt, int valid,
-                                            const uint32_t (&qf)[8][2], float sl, int lane) {
-    const int r = lane >> 2, c = lane & 3;
-
-    // ---- S^T (16 tokens x 8 heads) = K (16 x 128) . Q^T ----
+__device__ __forceinline__ void page_logits(float (&x)[4], uint32_t kt, int valid, const uint32_t (&qf)[8][2],
+                                            float sl, int lane) {
+    const int r = lane >> 2;
     // Two independent accumulators (even and odd k-steps) halve the chain of
     // dependent tensor-core ops; their sum is the contraction over all channels.
     float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
-        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-        if constexpr (!kFp8) {
+    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+    if constexpr (!kFp8) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int chunk = (kk & 3) * 2 + (lane >> 4);
-                const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(addr, a0, a1, a2, a3);
-                mma_16816(sacc[kk & 1], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-            }
-        } else {
+        for (int kk = 0; kk < 8; ++kk) {
+            const int chunk = (kk & 3) * 2 + (lane >> 4);
+            const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+            mma_16816(sacc[kk & 1], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+        }
+    } else {
 #pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                const int chunk = 2 * J + (lane >> 4);
-                const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
-                uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
-                ldsm_x4(addr, r0, r1, r2, r3);
-                mma_16816(sacc[0], e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
-                          e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
-                          qf[2 * J][0], qf[2 * J][1]);
-                mma_16816(sacc[1], e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
-                          e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
-                          qf[2 * J + 1][0], qf[2 * J + 1][1]);
-            }
+        for (int J = 0; J < 4; ++J) {
+            const int chunk = 2 * J + (lane >> 4);
+            const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
+            uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
+            ldsm_x4(addr, r0, r1, r2, r3);
+            mma_16816(sacc[0], e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
+                      e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
+                      qf[2 * J][0], qf[2 * J][1]);
+            mma_16816(sacc[1], e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
+                      e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
+                      qf[2 * J + 1][0], qf[2 * J + 1][1]);
         }
     }
-
-    // ---- online softmax over this page's tokens (rows r, r+8) ----
-    float x0 = (sacc[0][0] + sacc[1][0]) * sl, x1 = (sacc[0][1] + sacc[1][1]) * sl;
-    float x2 = (sacc[0][2] + sacc[1][2]) * sl, x3 = (sacc[0][3] + sacc[1][3]) * sl;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = (sacc[0][k] + sacc[1][k]) * sl;
     if (valid < kPageRows) {                    // rows past the context: excluded
-        if (r >= valid) x0 = x1 = -INFINITY;
-        if (r + 8 >= valid) x2 = x3 = -INFINITY;
+        if (r >= valid) x[0] = x[1] = -INFINITY;
+        if (r + 8 >= valid) x[2] = x[3] = -INFINITY;
     }
-    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-    }
-    const float mn0 = fmaxf(st.m0, bm0), mn1 = fmaxf(st.m1, bm1);
-    const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
-    st.m0 = mn0;
-    st.m1 = mn1;
-    const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
-    const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
-    st.l0 = st.l0 * al0 + (p0 + p2);
-    st.l1 = st.l1 * al1 + (p1 + p3);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        st.o[i][0] *= al0; st.o[i][1] *= al1; st.o[i][2] *= al0; st.o[i][3] *= al1;
-    }
-    // P^T as the B operand: transpose the (token x head) accumulator layout.
-    const uint32_t pb0 = movmatrix_trans(pack_half2(p0, p1));   // tokens 0..7
-    const uint32_t pb1 = movmatrix_trans(pack_half2(p2, p3));   // tokens 8..15
+}
 
-    // ---- O^T (128 ch x 8 heads) += V^T (128 x 16 tokens) . P^T ----
+// O^T (128 ch x 8 heads) += V^T (128 x 16 tokens) . P^T of one page, P^T given
+// as the B operand (pb0: tokens 0..7, pb1: tokens 8..15); V tile at shared
+// address vt, rows at or past `valid` read as zero.
+template <bool kFp8>
+__device__ __forceinline__ void page_pv(float (&o)[8][4], uint32_t vt, int valid, uint32_t pb0, uint32_t pb1,
+                                        int lane) {
+    const int r = lane >> 2, c = lane & 3;
     if constexpr (!kFp8) {
         uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // zero V of excluded rows
         if (valid < kPageRows) {
@@ -150,7 +131,7 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
             const uint32_t addr = vt + (i >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4_trans(addr, a0, a1, a2, a3);
-            mma_16816(st.o[i], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
+            mma_16816(o[i], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
         }
     } else {
         // lane (r, c) reads channels 16r..16r+15 of token rows 2c, 2c+1, 2c+8, 2c+9
@@ -172,10 +153,80 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
             const uint32_t sel = (i & 1) ? 0x7362u : 0x5140u;
             const uint32_t top = prmt(wa[i >> 1], wb[i >> 1], sel);   // tokens 2c, 2c+1
             const uint32_t bot = prmt(wc[i >> 1], wd[i >> 1], sel);   // tokens 2c+8, 2c+9
-            mma_16816(st.o[i], e4m3x2_to_half2(top), e4m3x2_to_half2(top >> 16),
+            mma_16816(o[i], e4m3x2_to_half2(top), e4m3x2_to_half2(top >> 16),
                       e4m3x2_to_half2(bot), e4m3x2_to_half2(bot >> 16), pb0, pb1);
         }
     }
+}
+
+// Online-softmax step of `st` over the logits of `kPages` pages (16 tokens
+// each): new running max, rescale of l and O by exp2(m_old - m_new), the
+// probabilities of the new tokens added to l, and P^T of each page as the
+// B operand (pb[2 * page], pb[2 * page + 1]).
+template <int kPages>
+__device__ __forceinline__ void softmax_step(WarpState& st, const float (&x)[kPages][4], uint32_t (&pb)[2 * kPages]) {
+    float bm0 = -INFINITY, bm1 = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kPages; ++q) {
+        bm0 = fmaxf(bm0, fmaxf(x[q][0], x[q][2]));
+        bm1 = fmaxf(bm1, fmaxf(x[q][1], x[q][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+    }
+    const float mn0 = fmaxf(st.m0, bm0), mn1 = fmaxf(st.m1, bm1);
+    const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
+    st.m0 = mn0;
+    st.m1 = mn1;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < kPages; ++q) {
+        const float p0 = fast_exp2(x[q][0] - mn0), p1 = fast_exp2(x[q][1] - mn1);
+        const float p2 = fast_exp2(x[q][2] - mn0), p3 = fast_exp2(x[q][3] - mn1);
+        s0 += p0 + p2;
+        s1 += p1 + p3;
+        // P^T as the B operand: transpose the (token x head) accumulator layout.
+        pb[2 * q] = movmatrix_trans(pack_half2(p0, p1));       // tokens 0..7
+        pb[2 * q + 1] = movmatrix_trans(pack_half2(p2, p3));   // tokens 8..15
+    }
+    st.l0 = st.l0 * al0 + s0;
+    st.l1 = st.l1 * al1 + s1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        st.o[i][0] *= al0; st.o[i][1] *= al1; st.o[i][2] *= al0; st.o[i][3] *= al1;
+    }
+}
+
+// Online-softmax update of `st` with one page: K tile at shared address kt,
+// V tile at vt, the first `valid` rows live. `sl` = softmax scale * log2(e)
+// (* k_scale for FP8).
+template <bool kFp8>
+__device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t vt, int valid,
+                                            const uint32_t (&qf)[8][2], float sl, int lane) {
+    float x[1][4];
+    page_logits<kFp8>(x[0], kt, valid, qf, sl, lane);
+    uint32_t pb[2];
+    softmax_step<1>(st, x, pb);
+    page_pv<kFp8>(st.o, vt, valid, pb[0], pb[1], lane);
+}
+
+// The same update with two consecutive pages of one segment in one softmax
+// step: page A (all 16 rows live) at ka/va, page B (the first valid_b rows
+// live) at kb/vb. Their logits are independent tensor-core chains and the
+// max, rescale and shuffles are paid once for 32 tokens.
+template <bool kFp8>
+__device__ __forceinline__ void attend_page_pair(WarpState& st, uint32_t ka, uint32_t va, uint32_t kb,
+                                                 uint32_t vb, int valid_b, const uint32_t (&qf)[8][2], float sl,
+                                                 int lane) {
+    float x[2][4];
+    page_logits<kFp8>(x[0], ka, kPageRows, qf, sl, lane);
+    page_logits<kFp8>(x[1], kb, valid_b, qf, sl, lane);
+    uint32_t pb[4];
+    softmax_step<2>(st, x, pb);
+    page_pv<kFp8>(st.o, va, kPageRows, pb[0], pb[1], lane);
+    page_pv<kFp8>(st.o, vb, valid_b, pb[2], pb[3], lane);
 }
 
 }  // namespace pkv

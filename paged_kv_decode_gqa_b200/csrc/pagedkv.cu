@@ -27,20 +27,26 @@ constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
 constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 
 // Balanced streaming kernel: worker warps per CTA and page slots per worker
-// ring (f16 pages are 8 KiB, FP8 pages 4 KiB). The defaults -- 8 workers with
-// 3 f16 (6 FP8) slots each, 192 KiB of ring, one CTA per SM -- measured best
-// or near best on every benchmark workload among 4x3 (two CTAs per SM), 4x6,
-// 6x4 and 8x3; the macros exist for tuning builds.
-#ifndef PKV_BAL_WARPS
-#define PKV_BAL_WARPS 8
+// ring (f16 pages are 8 KiB, FP8 pages 4 KiB), one CTA per SM (255 registers a
+// thread). Measured best on the benchmark workloads with two-page softmax
+// steps: f16 6 workers x 3 slots (144 KiB of ring; 8 x 3 took 17% longer on
+// the 1.5B-shaped step and 25% on the skewed one, 7B-shaped steps were within
+// 2% for 5..8 workers), FP8 8 workers x 4 slots (64 KiB; 8 x 6 and 7 x 6 were
+// slower). The macros exist for tuning builds.
+#ifndef PKV_BAL_WARPS_F16
+#define PKV_BAL_WARPS_F16 6
+#endif
+#ifndef PKV_BAL_WARPS_FP8
+#define PKV_BAL_WARPS_FP8 8
 #endif
 #ifndef PKV_BAL_STAGES_F16
 #define PKV_BAL_STAGES_F16 3
 #endif
 #ifndef PKV_BAL_STAGES_FP8
-#define PKV_BAL_STAGES_FP8 6
+#define PKV_BAL_STAGES_FP8 4
 #endif
-constexpr int kBalWarps = PKV_BAL_WARPS;
+constexpr int kBalWarpsF16 = PKV_BAL_WARPS_F16;
+constexpr int kBalWarpsFp8 = PKV_BAL_WARPS_FP8;
 constexpr int kBalStagesF16 = PKV_BAL_STAGES_F16;
 constexpr int kBalStagesFp8 = PKV_BAL_STAGES_FP8;
 constexpr int kBalMaxBatch = 8192;        // unit-order tables must fit in shared memory
@@ -160,12 +166,15 @@ pkv_status launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& mk, co
                ? PKV_OK : PKV_ERR_CUDA;
 }
 
+int bal_warps(bool fp8) { return fp8 ? kBalWarpsFp8 : kBalWarpsF16; }
+
 template <bool kFp8>
-using BalShape = pkv::BalancedShape<kFp8, kBalWarps, kFp8 ? kBalStagesFp8 : kBalStagesF16>;
+using BalShape = pkv::BalancedShape<kFp8, kFp8 ? kBalWarpsFp8 : kBalWarpsF16, kFp8 ? kBalStagesFp8 : kBalStagesF16>;
 
 template <bool kFp8, bool kFuse = false>
 auto balanced_kernel() {
-    return pkv::decode_balanced_kernel<kFp8, kBalWarps, kFp8 ? kBalStagesFp8 : kBalStagesF16, kFuse>;
+    return pkv::decode_balanced_kernel<kFp8, kFp8 ? kBalWarpsFp8 : kBalWarpsF16,
+                                       kFp8 ? kBalStagesFp8 : kBalStagesF16, kFuse>;
 }
 
 // Persistent grid of the balanced kernel for batch B on the current device:
@@ -225,7 +234,7 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
                            int32_t max_context_len, float softmax_scale, float k_scale, float v_scale,
                            void* workspace, size_t workspace_bytes, bool overlap_previous,
                            cudaStream_t st) {
-    const BalancedLayout bl = balanced_layout((int64_t)grid * kBalWarps, batch, Hkv);
+    const BalancedLayout bl = balanced_layout((int64_t)grid * bal_warps(fp8), batch, Hkv);
     if (!workspace || workspace_bytes < bl.total) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -260,7 +269,7 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, Hkv))
         return PKV_ERR_CUDA;
     const bool fuse = k_new != nullptr;
-    const dim3 g(grid), blk(BalShape<false>::kThreads);
+    const dim3 g(grid), blk(fp8 ? BalShape<true>::kThreads : BalShape<false>::kThreads);
     cudaError_t e;
     if (fp8)
         e = fuse ? launch_pdl(balanced_kernel<true, true>(), g, blk, BalShape<true>::smem_bytes(batch), st, mk, mv, bp)
@@ -382,17 +391,25 @@ size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
     if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim ||
         max_context_len < 0 || partition_tokens < PKV_PARTITION_AUTO)
         return 0;
-    if (partition_tokens == PKV_PARTITION_AUTO) {
-        const int64_t max_blocks = std::max(1, (max_context_len + kPageRows - 1) / kPageRows);
-        const int grid = use_balanced(batch, num_kv_heads, max_blocks)
-                             ? std::max(balanced_grid<false>(batch), balanced_grid<true>(batch)) : 0;
-        if (grid > 0) return balanced_layout((int64_t)grid * kBalWarps, batch, num_kv_heads).total;
-        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
-                                                              kPageRows, 0);
-    }
-    if (partition_tokens == 0) return 0;
-    const int64_t nparts = std::max<int64_t>(1, (max_context_len + partition_tokens - 1) / partition_tokens);
-    return workspace_layout(batch, num_q_heads, num_kv_heads, nparts).total;
+    auto fixed_size = [&](int32_t P) -> size_t {
+        if (P == 0) return 0;
+        const int64_t nparts = std::max<int64_t>(1, (max_context_len + P - 1) / P);
+        return workspace_layout(batch, num_q_heads, num_kv_heads, nparts).total;
+    };
+    if (partition_tokens != PKV_PARTITION_AUTO) return fixed_size(partition_tokens);
+    // AUTO: the cache type is not an argument, so cover both. Each runs the
+    // balanced plan if its tables fit, else the suggested fixed partitions.
+    const int64_t max_blocks = std::max(1, (max_context_len + kPageRows - 1) / kPageRows);
+    const bool balanced = use_balanced(batch, num_kv_heads, max_blocks);
+    const int g16 = balanced ? balanced_grid<false>(batch) : 0;
+    const int g8 = balanced ? balanced_grid<true>(batch) : 0;
+    size_t need = 0;
+    if (g16 > 0) need = std::max(need, balanced_layout((int64_t)g16 * kBalWarpsF16, batch, num_kv_heads).total);
+    if (g8 > 0) need = std::max(need, balanced_layout((int64_t)g8 * kBalWarpsFp8, batch, num_kv_heads).total);
+    if (g16 <= 0 || g8 <= 0)
+        need = std::max(need, fixed_size(paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
+                                                                            kPageRows, 0)));
+    return need;
 }
 
 int32_t paged_gqa_decode_suggest_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,

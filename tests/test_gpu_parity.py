@@ -350,6 +350,17 @@ def test_auto_one_sequence_split_over_many_workers():
     assert_attention_close(host(r.attention(AUTO)), r.oracle(), "auto long")
 
 
+def test_auto_fp8_batch_beyond_its_tables_falls_back():
+    """4000 sequences: the FP8 balanced tables no longer fit in shared memory while the f16
+    ones do, so FP8 runs fixed partitions inside the workspace sized for the automatic plan."""
+    w = W.with_sizes(W.WORKLOADS["fp8-e4m3"], B=4000, num_blocks=12000, ctx=("uniform", 1, 40))
+    r = _run(w, 18)
+    seqs = np.arange(0, w.B, 20)
+    out = host(r.attention(AUTO))
+    assert_attention_close(out[seqs], r.oracle(seqs=seqs), "auto fp8 fallback")
+    assert pkv.pkv_device_error() == 0
+
+
 def test_auto_batch_beyond_balanced_tables_falls_back():
     w = W.with_sizes(W.WORKLOADS["qwen2.5-1.5b"], B=9000, num_blocks=20000, ctx=("uniform", 1, 40))
     r = _run(w, 16)
