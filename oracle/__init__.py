@@ -63,6 +63,15 @@ def _load():
         lib.oracle_paged_gqa_decode.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                                 i32, i32, f32, i32, f32, f32, i32]
         lib.oracle_paged_gqa_decode.restype = i32
+        lib.oracle_paged_kv_cache_write_scaled.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
+        lib.oracle_paged_kv_cache_write_scaled.restype = i32
+        lib.oracle_paged_gqa_decode_scaled.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                       i32, i32, f32, i32, P, P, i32]
+        lib.oracle_paged_gqa_decode_scaled.restype = i32
+        lib.oracle_absmax_f16.argtypes = [P, i64, i32, i32, i32, P]
+        lib.oracle_absmax_f16.restype = None
+        lib.oracle_fp8_scale_from_amax.argtypes = [f32]
+        lib.oracle_fp8_scale_from_amax.restype = f32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -114,12 +123,23 @@ def quantize_e4m3(x_f16: np.ndarray, scale: float) -> np.ndarray:
     return out
 
 
+def _head_scales(scale, Hkv):
+    """A scale argument as float32[Hkv]: per KV head if it has Hkv entries, else one per-tensor value."""
+    a = np.asarray(scale, dtype=np.float32).ravel()
+    if a.size == 1:
+        return np.full(Hkv, a[0], dtype=np.float32), False
+    if a.size != Hkv:
+        raise ValueError("a per-head scale needs one value per KV head")
+    return np.ascontiguousarray(a), True
+
+
 def paged_kv_cache_write(k_new, v_new, k_cache, v_cache, slot_mapping, *,
-                         kv_dtype: str = "f16", k_scale: float = 1.0, v_scale: float = 1.0):
+                         kv_dtype: str = "f16", k_scale=1.0, v_scale=1.0):
     """In-place cache write on NumPy copies of the caches (reshape_and_cache).
 
     k_new, v_new: [T, Hkv, D] float16. k_cache, v_cache: [NB, bs, Hkv, D],
     float16 or uint8 (FP8 codes). slot_mapping: [T] int64, negative = skip.
+    k_scale / v_scale: one per-tensor value, or one value per KV head.
     """
     k_new = _c(k_new, np.float16)
     v_new = _c(v_new, np.float16)
@@ -132,20 +152,28 @@ def paged_kv_cache_write(k_new, v_new, k_cache, v_cache, slot_mapping, *,
     slots = _c(slot_mapping, np.int64)
     T, Hkv, D = k_new.shape
     NB, bs = k_cache.shape[0], k_cache.shape[1]
-    rc = _load().oracle_paged_kv_cache_write(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
-                                             _ptr(slots), T, Hkv, D, NB, bs, int(fp8),
-                                             ctypes.c_float(k_scale), ctypes.c_float(v_scale))
+    ks, k_ph = _head_scales(k_scale, Hkv)
+    vs, v_ph = _head_scales(v_scale, Hkv)
+    if k_ph or v_ph:
+        rc = _load().oracle_paged_kv_cache_write_scaled(_ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                                        _ptr(v_cache), _ptr(slots), T, Hkv, D, NB, bs,
+                                                        int(fp8), _ptr(ks), _ptr(vs))
+    else:
+        rc = _load().oracle_paged_kv_cache_write(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                                 _ptr(slots), T, Hkv, D, NB, bs, int(fp8),
+                                                 ctypes.c_float(ks[0]), ctypes.c_float(vs[0]))
     if rc != 0:
         raise ValueError("slot outside the pool")
 
 
 def paged_gqa_decode(q, k_cache, v_cache, block_tables, context_lens, softmax_scale, *,
-                     kv_dtype: str = "f16", k_scale: float = 1.0, v_scale: float = 1.0,
+                     kv_dtype: str = "f16", k_scale=1.0, v_scale=1.0,
                      partition_tokens: int = 0, return_lse: bool = False):
     """Decode attention in float64 through the block tables.
 
     q: [B, Hq, D] float16. k_cache, v_cache: [NB, bs, Hkv, D] float16 or
     uint8 (FP8). block_tables: [B, max_blocks] int32. context_lens: [B] int32.
+    k_scale / v_scale (FP8): one per-tensor value, or one value per KV head.
     Returns out [B, Hq, D] float64 (and lse [B, Hq] float64 if asked).
     """
     q = _c(q, np.float16)
@@ -161,13 +189,45 @@ def paged_gqa_decode(q, k_cache, v_cache, block_tables, context_lens, softmax_sc
         raise ValueError("shape mismatch")
     out = np.zeros((B, Hq, D), dtype=np.float64)
     lse = np.zeros((B, Hq), dtype=np.float64)
-    rc = _load().oracle_paged_gqa_decode(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                         _ptr(bt), _ptr(cl), B, Hq, Hkv, D, bs, bt.shape[1], NB,
-                                         ctypes.c_float(softmax_scale), int(fp8),
-                                         ctypes.c_float(k_scale), ctypes.c_float(v_scale),
-                                         int(partition_tokens))
+    ks, k_ph = _head_scales(k_scale, Hkv)
+    vs, v_ph = _head_scales(v_scale, Hkv)
+    if k_ph or v_ph:
+        rc = _load().oracle_paged_gqa_decode_scaled(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache),
+                                                    _ptr(v_cache), _ptr(bt), _ptr(cl), B, Hq, Hkv, D, bs,
+                                                    bt.shape[1], NB, ctypes.c_float(softmax_scale),
+                                                    int(fp8), _ptr(ks), _ptr(vs), int(partition_tokens))
+    else:
+        rc = _load().oracle_paged_gqa_decode(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                             _ptr(bt), _ptr(cl), B, Hq, Hkv, D, bs, bt.shape[1], NB,
+                                             ctypes.c_float(softmax_scale), int(fp8),
+                                             ctypes.c_float(ks[0]), ctypes.c_float(vs[0]),
+                                             int(partition_tokens))
     if rc == -1:
         raise ValueError("block table entry outside the pool")
     if rc != 0:
         raise ValueError("bad head counts or context length")
     return (out, lse) if return_lse else out
+
+
+def absmax_f16(x, per_head: bool):
+    """Largest |x| over the non-NaN elements of x [rows, Hkv, D] float16: float32[Hkv]
+    per KV head, or float32[1] over the tensor; 0 where nothing counts."""
+    x = _c(x, np.float16)
+    if x.ndim != 3:
+        raise ValueError("x must be [rows, Hkv, D]")
+    rows, Hkv, D = x.shape
+    out = np.zeros(Hkv if per_head else 1, dtype=np.float32)
+    _load().oracle_absmax_f16(_ptr(x), rows, Hkv, D, int(bool(per_head)), _ptr(out))
+    return out
+
+
+def fp8_scale_from_amax(amax):
+    """E4M3 cache scale(s) fp32(amax) / 448 (fp32 division); 1 where amax is 0."""
+    a = np.asarray(amax, dtype=np.float32).ravel()
+    lib = _load()
+    return np.array([lib.oracle_fp8_scale_from_amax(float(v)) for v in a], dtype=np.float32)
+
+
+def fp8_scales(x, per_head: bool):
+    """Scales an E4M3 cache would use for the data x [rows, Hkv, D] float16."""
+    return fp8_scale_from_amax(absmax_f16(x, per_head))

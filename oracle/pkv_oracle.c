@@ -31,7 +31,12 @@
  *      decoded value by the scale;
  *   R6 split-KV partitions are aligned to multiples of partition_tokens in
  *      logical token order and are merged with the log-sum-exp rule;
- *   R7 a negative slot in the cache write means "skip this token".
+ *   R7 a negative slot in the cache write means "skip this token";
+ *   R8 (FP8 variants) a scale may also be given per KV head, scale[h]
+ *      replacing the per-tensor scale for every element of head h; a scale
+ *      computed from data is fp32(amax) / 448 divided in fp32, amax being
+ *      the largest |x| over the non-NaN elements (per head, or over the
+ *      whole tensor), and 1 when that maximum is 0 (or no element counts).
  *
  * Build: gcc -O2 -fopenmp -fPIC -shared -ffp-contract=off (no fast-math).
  */
@@ -127,13 +132,14 @@ void oracle_quantize_e4m3(const uint16_t* x, int64_t n, float scale, uint8_t* ou
 /* reshape_and_cache: token i of this step goes to slot s = slot_mapping[i],
  * i.e. block s / block_size, row s % block_size (R2); for every KV head h
  * and channel d:  k_cache[blk][row][h][d] = k_new[i][h][d], same for V.
- * FP8 caches store e4m3(k_new / k_scale) (R5). Negative slots are skipped
- * (R7). Returns 0, or -1 if a slot lies outside the pool. */
-int oracle_paged_kv_cache_write(const uint16_t* k_new, const uint16_t* v_new,
-                                void* k_cache, void* v_cache,
-                                const int64_t* slot_mapping, int T, int Hkv, int D,
-                                int num_blocks, int block_size, int kv_fp8,
-                                float k_scale, float v_scale) {
+ * FP8 caches store e4m3(k_new / k_scales[h]) (R5, R8: one scale per KV head).
+ * Negative slots are skipped (R7). Returns 0, or -1 if a slot lies outside
+ * the pool. */
+int oracle_paged_kv_cache_write_scaled(const uint16_t* k_new, const uint16_t* v_new,
+                                       void* k_cache, void* v_cache,
+                                       const int64_t* slot_mapping, int T, int Hkv, int D,
+                                       int num_blocks, int block_size, int kv_fp8,
+                                       const float* k_scales, const float* v_scales) {
     for (int i = 0; i < T; ++i) {
         int64_t s = slot_mapping[i];
         if (s < 0) continue;
@@ -144,8 +150,8 @@ int oracle_paged_kv_cache_write(const uint16_t* k_new, const uint16_t* v_new,
                 int64_t src = ((int64_t)i * Hkv + h) * D + d;
                 int64_t dst = ((blk * block_size + row) * Hkv + h) * D + d;
                 if (kv_fp8) {
-                    ((uint8_t*)k_cache)[dst] = quantize_one(k_new[src], k_scale);
-                    ((uint8_t*)v_cache)[dst] = quantize_one(v_new[src], v_scale);
+                    ((uint8_t*)k_cache)[dst] = quantize_one(k_new[src], k_scales[h]);
+                    ((uint8_t*)v_cache)[dst] = quantize_one(v_new[src], v_scales[h]);
                 } else {
                     ((uint16_t*)k_cache)[dst] = k_new[src];
                     ((uint16_t*)v_cache)[dst] = v_new[src];
@@ -156,10 +162,51 @@ int oracle_paged_kv_cache_write(const uint16_t* k_new, const uint16_t* v_new,
     return 0;
 }
 
+/* The same write with one per-tensor scale: every KV head uses it (R5). */
+int oracle_paged_kv_cache_write(const uint16_t* k_new, const uint16_t* v_new,
+                                void* k_cache, void* v_cache,
+                                const int64_t* slot_mapping, int T, int Hkv, int D,
+                                int num_blocks, int block_size, int kv_fp8,
+                                float k_scale, float v_scale) {
+    float* ks = (float*)malloc(sizeof(float) * (size_t)(Hkv > 0 ? Hkv : 1));
+    float* vs = (float*)malloc(sizeof(float) * (size_t)(Hkv > 0 ? Hkv : 1));
+    for (int h = 0; h < Hkv; ++h) { ks[h] = k_scale; vs[h] = v_scale; }
+    int rc = oracle_paged_kv_cache_write_scaled(k_new, v_new, k_cache, v_cache, slot_mapping, T, Hkv,
+                                                D, num_blocks, block_size, kv_fp8, ks, vs);
+    free(ks);
+    free(vs);
+    return rc;
+}
+
+/* ------------------------------------------------------------- FP8 scales */
+
+/* Largest |x| of the non-NaN elements of x[rows][Hkv][D] (binary16), per KV
+ * head (per_head != 0: amax[h], h < Hkv) or over the whole tensor (amax[0]);
+ * 0 when nothing counts (R8). */
+void oracle_absmax_f16(const uint16_t* x, int64_t rows, int Hkv, int D, int per_head, float* amax) {
+    int n_out = per_head ? Hkv : 1;
+    for (int h = 0; h < n_out; ++h) amax[h] = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int h = 0; h < Hkv; ++h)
+            for (int d = 0; d < D; ++d) {
+                double v = fabs(oracle_f16_to_f64(x[(r * Hkv + h) * D + d]));
+                if (isnan(v)) continue;
+                float* a = &amax[per_head ? h : 0];
+                if (v > (double)*a) *a = (float)v;      /* exact: a binary16 magnitude is an fp32 */
+            }
+}
+
+/* Scale of an E4M3 cache for a given amax (R8): fp32 division by 448, so the
+ * largest magnitude maps onto the largest finite code; 1 for amax 0. */
+float oracle_fp8_scale_from_amax(float amax) {
+    if (!(amax > 0.0f)) return 1.0f;
+    return amax / 448.0f;                           /* IEEE fp32 division */
+}
+
 /* --------------------------------------------------------- decode attention */
 
 /* Cache element (token row `slot` of the pool, KV head g, channel d) as f64:
- * f16 directly, FP8 as decoded value times the per-tensor scale (R5). */
+ * f16 directly, FP8 as decoded value times the scale of KV head g (R5, R8). */
 static double cache_elem(const void* cache, int kv_fp8, double scale,
                          int64_t slot, int Hkv, int D, int g, int d) {
     int64_t idx = (slot * Hkv + g) * D + d;
@@ -175,9 +222,10 @@ static int attend_range(double* m_out, double* l_out, double* o, double* s,
                         const uint16_t* q, const void* k_cache, const void* v_cache,
                         const int32_t* bt_row, int b, int h, int Hq, int Hkv, int D,
                         int block_size, int num_blocks, double scale, int kv_fp8,
-                        double k_scale, double v_scale, int t0, int t1) {
+                        const float* k_scales, const float* v_scales, int t0, int t1) {
     int G = Hq / Hkv;
     int g = h / G;                                  /* R1 */
+    double k_scale = kv_fp8 ? (double)k_scales[g] : 1.0, v_scale = kv_fp8 ? (double)v_scales[g] : 1.0;
     const uint16_t* qh = q + ((int64_t)b * Hq + h) * D;
     /* logits s_t = scale * sum_d q[d] k_t[d], gathering k_t through the table */
     double m = -INFINITY;
@@ -215,12 +263,13 @@ static int attend_range(double* m_out, double* l_out, double* o, double* s,
  * lse (optional, [B][Hq]) receives the log-sum-exp of the logits: m + ln l,
  * or M + ln(sum_p w_p) when split; -inf for an empty context (R4).
  * Returns 0, -1 for a table entry outside the pool, -2 for a bad length. */
-int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
-                            const void* k_cache, const void* v_cache,
-                            const int32_t* block_tables, const int32_t* context_lens,
-                            int B, int Hq, int Hkv, int D, int block_size,
-                            int max_blocks_per_seq, int num_blocks, float softmax_scale,
-                            int kv_fp8, float k_scale, float v_scale, int partition_tokens) {
+int oracle_paged_gqa_decode_scaled(double* out, double* lse, const uint16_t* q,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int B, int Hq, int Hkv, int D, int block_size,
+                                   int max_blocks_per_seq, int num_blocks, float softmax_scale,
+                                   int kv_fp8, const float* k_scales, const float* v_scales,
+                                   int partition_tokens) {
     if (Hkv <= 0 || Hq % Hkv != 0) return -2;
     int status = 0;
 #pragma omp parallel for collapse(2) schedule(dynamic)
@@ -248,8 +297,7 @@ int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
                 int t0 = p * P, t1 = (p + 1) * P < L ? (p + 1) * P : L;
                 if (attend_range(&mp[p], &lp[p], &op[(int64_t)p * D], s, q, k_cache, v_cache,
                                  bt_row, b, h, Hq, Hkv, D, block_size, num_blocks,
-                                 (double)softmax_scale, kv_fp8, (double)k_scale,
-                                 (double)v_scale, t0, t1))
+                                 (double)softmax_scale, kv_fp8, k_scales, v_scales, t0, t1))
                     bad = 1;
             }
             if (bad) {
@@ -274,6 +322,25 @@ int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
         }
     }
     return status;
+}
+
+/* The same attention with one per-tensor scale for K and one for V (R5). */
+int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
+                            const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int B, int Hq, int Hkv, int D, int block_size,
+                            int max_blocks_per_seq, int num_blocks, float softmax_scale,
+                            int kv_fp8, float k_scale, float v_scale, int partition_tokens) {
+    if (Hkv <= 0) return -2;
+    float* ks = (float*)malloc(sizeof(float) * (size_t)Hkv);
+    float* vs = (float*)malloc(sizeof(float) * (size_t)Hkv);
+    for (int h = 0; h < Hkv; ++h) { ks[h] = k_scale; vs[h] = v_scale; }
+    int rc = oracle_paged_gqa_decode_scaled(out, lse, q, k_cache, v_cache, block_tables, context_lens,
+                                            B, Hq, Hkv, D, block_size, max_blocks_per_seq, num_blocks,
+                                            softmax_scale, kv_fp8, ks, vs, partition_tokens);
+    free(ks);
+    free(vs);
+    return rc;
 }
 
 /* Number of threads the OpenMP runtime would use for a parallel region. */
