@@ -247,6 +247,9 @@ def parse_args(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="two launches per step (cache write, then attention) instead of the fused step")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fp8-scales", default="tensor", choices=["tensor", "per-head"],
+                    help="FP8 workloads: per-tensor host scales, or per-KV-head scales computed on the "
+                         "device and passed to the device-scale entry points")
     ap.add_argument("--cpu-baseline-s", type=float, default=10.0)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args(argv)
@@ -320,15 +323,38 @@ def run_ours(args):
     touched = kv_bytes(lens, Hkv, D, 1 if fp8 else 2)
     R = max(1, min(16, -(-4 * L2_BYTES // max(touched, 1))))
     k16, v16 = t(x["k_pool"]), t(x["v_pool"])
+    per_head = fp8 and args.fp8_scales == "per-head"
+    scales_kernel = None
     if fp8:                                        # quantise the pool with the library's cache write
         kq = torch.empty(k16.shape, dtype=torch.uint8, device=device)
         vq = torch.empty_like(kq)
         n_rows = w.num_blocks * bs
-        pkv.paged_kv_cache_write(k16.view(n_rows, Hkv, D), v16.view(n_rows, Hkv, D), kq, vq,
-                                 torch.arange(n_rows, dtype=torch.int64, device=device),
-                                 kv_dtype="fp8", k_scale=ks, v_scale=vs)
+        rows_k, rows_v = k16.view(n_rows, Hkv, D), v16.view(n_rows, Hkv, D)
+        all_slots = torch.arange(n_rows, dtype=torch.int64, device=device)
+        if per_head:
+            # per-KV-head scales computed on the device from the pool (its free rows are NaN and
+            # do not count); the scales kernel is timed over the K pool
+            ks_t = torch.empty(Hkv, dtype=torch.float32, device=device)
+            vs_t = torch.empty(Hkv, dtype=torch.float32, device=device)
+            for _ in range(3):
+                pkv.paged_kv_fp8_scales(rows_k, ks_t, per_head=True, stream=stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 10
+            e0.record(stream)
+            for _ in range(reps):
+                pkv.paged_kv_fp8_scales(rows_k, ks_t, per_head=True, stream=stream)
+            e1.record(stream)
+            pkv.paged_kv_fp8_scales(rows_v, vs_t, per_head=True, stream=stream)
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1000 / reps
+            nbytes = rows_k.numel() * 2
+            scales_kernel = {"input_bytes": nbytes, "us": us, "gbs": nbytes / us / 1e3,
+                             "what": "paged_kv_fp8_scales, per KV head, over the f16 K pool (memset + 2 launches)"}
+            pkv.paged_kv_cache_write_fp8_scaled(rows_k, rows_v, kq, vq, all_slots, ks_t, vs_t, stream=stream)
+        else:
+            pkv.paged_kv_cache_write(rows_k, rows_v, kq, vq, all_slots, kv_dtype="fp8", k_scale=ks, v_scale=vs)
         base_k, base_v = kq, vq
-        del k16, v16
+        del k16, v16, rows_k, rows_v
     else:
         base_k, base_v = k16, v16
     pools = [(base_k, base_v)] + [(base_k.clone(), base_v.clone()) for _ in range(R - 1)]
@@ -339,25 +365,48 @@ def run_ours(args):
     fused = not args.unfused and P == pkv.PKV_PARTITION_AUTO
     step_flags = 0 if args.no_overlap else pkv.PKV_STEP_OVERLAP_PREVIOUS
 
+    # the library calls of one step, per-tensor scales or per-KV-head device scales
+    def write_call(kn, vn, kc, vc, sl):
+        if per_head:
+            pkv.paged_kv_cache_write_fp8_scaled(kn, vn, kc, vc, sl, ks_t, vs_t, stream=stream)
+        else:
+            pkv.paged_kv_cache_write(kn, vn, kc, vc, sl, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
+                                     stream=stream)
+
+    def step_call(qq, kn, vn, kc, vc, bb, cc, flags):
+        if per_head:
+            pkv.paged_gqa_decode_step_fp8_scaled(out, qq, kn, vn, kc, vc, bb, cc, ks_t, vs_t,
+                                                 max_context_len=max_len, softmax_scale=scale,
+                                                 workspace=ws, flags=flags, stream=stream)
+        else:
+            pkv.paged_gqa_decode_step(out, qq, kn, vn, kc, vc, bb, cc, max_context_len=max_len,
+                                      softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
+                                      workspace=ws, flags=flags, stream=stream)
+
+    def attention_call(qq, kc, vc, bb, cc):
+        if per_head:
+            pkv.paged_gqa_decode_attention_fp8_scaled(out, qq, kc, vc, bb, cc, ks_t, vs_t,
+                                                      max_context_len=max_len, softmax_scale=scale,
+                                                      partition_tokens=P, workspace=ws, stream=stream)
+        else:
+            pkv.paged_gqa_decode_attention(out, qq, kc, vc, bb, cc, max_context_len=max_len,
+                                           softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
+                                           v_scale=vs, partition_tokens=P, workspace=ws, stream=stream)
+
     def cache_write(i):
         if fused:                                  # the step kernel writes the new tokens itself
             return
         kc, vc = pools[i % R]
-        pkv.paged_kv_cache_write(k_new, v_new, kc, vc, slots, kv_dtype=w.kv_dtype, k_scale=ks,
-                                 v_scale=vs, stream=stream)
+        write_call(k_new, v_new, kc, vc, slots)
 
     def attention(i):
         kc, vc = pools[i % R]
         if fused:
             # consecutive steps read different pool replicas, so no launch writes
             # the pages the next one reads: the overlap promise holds
-            pkv.paged_gqa_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, max_context_len=max_len,
-                                      softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                      workspace=ws, flags=step_flags, stream=stream)
+            step_call(q, k_new, v_new, kc, vc, bt, cl, step_flags)
         else:
-            pkv.paged_gqa_decode_attention(out, q, kc, vc, bt, cl, max_context_len=max_len,
-                                           softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
-                                           v_scale=vs, partition_tokens=P, workspace=ws, stream=stream)
+            attention_call(q, kc, vc, bt, cl)
 
     # ---- warm-up: W eager steps (also sets kernel attributes and TMA maps) ----
     for i in range(args.warmup):
@@ -428,17 +477,10 @@ def run_ours(args):
                 d[k].copy_(h[k], non_blocking=True)
             kc, vc = pools[i % R]
             if fused:
-                pkv.paged_gqa_decode_step(out, d["q"], d["k_new"], d["v_new"], kc, vc, d["block_tables"],
-                                          d["context_lens"], max_context_len=max_len, softmax_scale=scale,
-                                          kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs, workspace=ws,
-                                          stream=stream)
+                step_call(d["q"], d["k_new"], d["v_new"], kc, vc, d["block_tables"], d["context_lens"], 0)
             else:
-                pkv.paged_kv_cache_write(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"],
-                                         kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs, stream=stream)
-                pkv.paged_gqa_decode_attention(out, d["q"], kc, vc, d["block_tables"], d["context_lens"],
-                                               max_context_len=max_len, softmax_scale=scale,
-                                               kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                               partition_tokens=P, workspace=ws, stream=stream)
+                write_call(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"])
+                attention_call(d["q"], kc, vc, d["block_tables"], d["context_lens"])
             out_h.copy_(out, non_blocking=True)
             stream.synchronize()
 
@@ -473,6 +515,7 @@ def run_ours(args):
             "pct_of_hbm_peak": 100.0 * value / peak,
             "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "head_dim": D,
                        "block_size": bs, "kv_dtype": w.kv_dtype, "context_lens": list(w.ctx),
+                       **({"fp8_scales": "per KV head, computed on the device"} if per_head else {}),
                        "partition_tokens": P, "parallelism": f"dp{world} (independent batches)",
                        "l2": f"inputs larger than L2: {R} KV pool replicas rotated, "
                              f"{R * touched / 2**20:.0f} MiB touched per cycle",
@@ -489,6 +532,8 @@ def run_ours(args):
             "gpu_launches": launches,
             "clocks": sampler.summary(wall0, wall1),
         }
+        if scales_kernel:
+            line["fp8_scales_kernel"] = scales_kernel
         if e2e:
             line["e2e"] = e2e
         if world == 1 and args.cpu_baseline_s > 0:

@@ -96,6 +96,8 @@ typedef enum {
                                           block read as zeros */
 #define PKV_DEVERR_SLOT          0x4u  /* a slot lay outside the pool; the token was skipped */
 #define PKV_DEVERR_WAIT_TIMEOUT  0x8u  /* an on-chip barrier wait ran out of its time limit */
+#define PKV_DEVERR_SCALE         0x10u /* a device-side FP8 scale was not positive and finite;
+                                          the results that used it are undefined */
 
 /*
  * paged_kv_cache_write -- reshape_and_cache.
@@ -279,6 +281,81 @@ pkv_status paged_gqa_decode_attention_static_workspace(
     int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
     int32_t max_context_len, float softmax_scale, int32_t kv_dtype,
     float k_scale, float v_scale, int32_t partition_tokens, void* stream);
+
+/*
+ * FP8 E4M3 caches with device-side scales (per tensor or per KV head).
+ *
+ * The pages name an FP8 E4M3 KV cache and no more ("rvLLM 소개"
+ * (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3). These entry points
+ * take the reading, stated beside each one, that a scale may be given per KV
+ * head and computed from data on the device, so that a step can be
+ * calibrated and captured in a CUDA graph without reading anything back to
+ * the host. Scale arrays are device pointers to float: one element when
+ * scales_per_head is 0 (per tensor), num_kv_heads elements (head h uses
+ * element h) when it is 1. They must hold positive finite values by the time
+ * the kernels run; a violation is flagged (PKV_DEVERR_SCALE), not checked on
+ * the host. Everything else is as for the per-tensor entry points above.
+ */
+
+/*
+ * paged_kv_fp8_scales -- E4M3 scales from data.
+ *
+ * x: [rows, num_kv_heads, head_dim] f16, contiguous (for example this step's
+ * new K, or the live rows of a cache being calibrated). Writes, on `stream`,
+ *   scales[h] = amax_h / 448   (fp32 IEEE division), or 1 when amax_h is 0,
+ * where amax_h is the largest |x| over the non-NaN elements of head h
+ * (scales_per_head == 1, scales[num_kv_heads]) or of the whole tensor
+ * (scales_per_head == 0, scales[1]); 448 is the largest finite E4M3 value,
+ * so the largest magnitude maps onto the largest code. Infinite elements give
+ * an infinite scale, which the FP8 kernels then flag. rows == 0 writes 1.
+ * scales_per_head == 1 needs num_kv_heads <= 1024. head_dim must be a
+ * multiple of 8 and x 16-byte aligned.
+ */
+pkv_status paged_kv_fp8_scales(const void* x, int64_t rows, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t scales_per_head, float* scales, void* stream);
+
+/*
+ * paged_kv_cache_write_fp8_scaled -- paged_kv_cache_write for an FP8 cache
+ * with device-side scales: head h of a token is stored as E4M3 codes of
+ * k_new / k_scales[h or 0] (v_new / v_scales[h or 0]), rounded to nearest
+ * even and saturated to +-448.
+ */
+pkv_status paged_kv_cache_write_fp8_scaled(const void* k_new, const void* v_new,
+                                           void* k_cache, void* v_cache,
+                                           const int64_t* slot_mapping,
+                                           int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                           int32_t num_blocks, int32_t block_size,
+                                           const float* k_scales, const float* v_scales,
+                                           int32_t scales_per_head, void* stream);
+
+/*
+ * paged_gqa_decode_attention_fp8_scaled -- paged_gqa_decode_attention on an
+ * FP8 cache whose element of KV head g dequantises as decode(byte) times
+ * k_scales[g or 0] (V: v_scales[g or 0]). All plans (single pass, fixed
+ * partitions, PKV_PARTITION_AUTO) and the same workspace rules apply.
+ */
+pkv_status paged_gqa_decode_attention_fp8_scaled(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+    int32_t max_context_len, float softmax_scale,
+    const float* k_scales, const float* v_scales, int32_t scales_per_head,
+    int32_t partition_tokens, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * paged_gqa_decode_step_fp8_scaled -- paged_gqa_decode_step on an FP8 cache
+ * with device-side scales: the new token is quantised with, and every element
+ * dequantised with, the scales of its KV head as above.
+ */
+pkv_status paged_gqa_decode_step_fp8_scaled(
+    void* out, const void* q, const void* k_new, const void* v_new,
+    void* k_cache, void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+    int32_t max_context_len, float softmax_scale,
+    const float* k_scales, const float* v_scales, int32_t scales_per_head,
+    void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,6 +39,15 @@ _SIGNATURES = {
     "paged_gqa_decode_attention_static_workspace": (
         [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _f32,
          _f32, _i32, _P], ctypes.c_int),
+    "paged_kv_fp8_scales": ([_P, ctypes.c_int64, _i32, _i32, _i32, _P, _P], ctypes.c_int),
+    "paged_kv_cache_write_fp8_scaled": ([_P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _P, _P, _i32, _P],
+                                        ctypes.c_int),
+    "paged_gqa_decode_attention_fp8_scaled": (
+        [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _P, _P, _i32, _i32,
+         _P, _sz, _P], ctypes.c_int),
+    "paged_gqa_decode_step_fp8_scaled": (
+        [_P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _P, _P, _i32,
+         _P, _sz, ctypes.c_uint32, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -73,7 +82,7 @@ PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_WORKSPACE, PKV_ERR_CUD
 PKV_KV_F16, PKV_KV_FP8_E4M3 = 0, 1
 PKV_PARTITION_AUTO = -1         # partition_tokens: the library's load-balanced plan
 PKV_STEP_OVERLAP_PREVIOUS = 0x1  # paged_gqa_decode_step flag (see include/pagedkv.h)
-DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT, DEVERR_SCALE = 0x1, 0x2, 0x4, 0x8, 0x10
 _KV_DTYPES = {"f16": PKV_KV_F16, "fp8": PKV_KV_FP8_E4M3}
 
 
@@ -235,3 +244,94 @@ def paged_gqa_decode_attention_static_workspace(out, q, k_cache, v_cache, block_
         B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(softmax_scale),
         kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), int(partition_tokens),
         _stream(stream)), "paged_gqa_decode_attention_static_workspace")
+
+
+# ----------------------------------------------------------------------------
+# FP8 E4M3 caches with device-side scales: one float per tensor, or one per KV
+# head (float32 CUDA tensors of 1 or Hkv elements).
+
+def _scales(k_scales, v_scales, Hkv):
+    _dense("k_scales", k_scales, "float32")
+    _dense("v_scales", v_scales, "float32")
+    n = k_scales.numel()
+    if v_scales.numel() != n or n not in (1, Hkv):
+        raise ValueError("k_scales and v_scales need 1 (per tensor) or num_kv_heads (per head) elements")
+    return int(n == Hkv and Hkv > 1)
+
+
+def paged_kv_fp8_scales(x, scales, *, per_head, stream=None) -> None:
+    """scales[h] = max|x[:, h, :]| / 448 over the non-NaN elements of x [rows, Hkv, D]
+    float16 (per KV head), or of all of x (per_head=False, one scale); 1 for a maximum of 0."""
+    _dense("x", x, "float16")
+    _dense("scales", scales, "float32")
+    rows, Hkv, D = x.shape
+    if scales.numel() != (Hkv if per_head else 1):
+        raise ValueError("scales needs num_kv_heads elements per head, else 1")
+    _check(load_library().paged_kv_fp8_scales(_ptr(x), rows, Hkv, D, int(bool(per_head)), _ptr(scales),
+                                              _stream(stream)), "paged_kv_fp8_scales")
+
+
+def paged_kv_cache_write_fp8_scaled(k_new, v_new, k_cache, v_cache, slot_mapping, k_scales, v_scales, *,
+                                    stream=None) -> None:
+    """paged_kv_cache_write into an FP8 cache, quantising head h with k_scales[h] / v_scales[h]
+    (or the single scale)."""
+    for n, t in (("k_new", k_new), ("v_new", v_new)):
+        _dense(n, t, "float16")
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _dense(n, t, "uint8")
+    _dense("slot_mapping", slot_mapping, "int64")
+    T, Hkv, D = k_new.shape
+    NB, bs = k_cache.shape[0], k_cache.shape[1]
+    per_head = _scales(k_scales, v_scales, Hkv)
+    _check(load_library().paged_kv_cache_write_fp8_scaled(
+        _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, NB, bs,
+        _ptr(k_scales), _ptr(v_scales), per_head, _stream(stream)), "paged_kv_cache_write_fp8_scaled")
+
+
+def paged_gqa_decode_attention_fp8_scaled(out, q, k_cache, v_cache, block_tables, context_lens, k_scales,
+                                          v_scales, *, max_context_len, softmax_scale, partition_tokens=0,
+                                          workspace=None, stream=None) -> None:
+    """paged_gqa_decode_attention on an FP8 cache whose KV head g dequantises with
+    k_scales[g] / v_scales[g] (or the single scale)."""
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    _dense("k_cache", k_cache, "uint8")
+    _dense("v_cache", v_cache, "uint8")
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    if workspace is not None:
+        _dense("workspace", workspace, "uint8", "float32", "int32")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    per_head = _scales(k_scales, v_scales, Hkv)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load_library().paged_gqa_decode_attention_fp8_scaled(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len), float(softmax_scale),
+        _ptr(k_scales), _ptr(v_scales), per_head, int(partition_tokens), _ptr(workspace), ws_bytes,
+        _stream(stream)), "paged_gqa_decode_attention_fp8_scaled")
+
+
+def paged_gqa_decode_step_fp8_scaled(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                                     k_scales, v_scales, *, max_context_len, softmax_scale, workspace=None,
+                                     flags=0, stream=None) -> None:
+    """paged_gqa_decode_step on an FP8 cache with device-side scales (per tensor or per KV head)."""
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    _dense("k_new", k_new, "float16")
+    _dense("v_new", v_new, "float16")
+    _dense("k_cache", k_cache, "uint8")
+    _dense("v_cache", v_cache, "uint8")
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    if workspace is not None:
+        _dense("workspace", workspace, "uint8", "float32", "int32")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    per_head = _scales(k_scales, v_scales, Hkv)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load_library().paged_gqa_decode_step_fp8_scaled(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
+        float(softmax_scale), _ptr(k_scales), _ptr(v_scales), per_head, _ptr(workspace), ws_bytes,
+        int(flags), _stream(stream)), "paged_gqa_decode_step_fp8_scaled")

@@ -2,7 +2,7 @@
 //
 // Each step's new key/value vectors ([T, Hkv, D] f16) go to the rows named by
 // slot_mapping (block = slot / block_size, row = slot % block_size), in f16 or
-// as OCP E4M3 codes with per-tensor scales. The pages describe the paged
+// as OCP E4M3 codes with per-tensor or per-KV-head scales. The pages describe the paged
 // cache ("rvLLM 소개" (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3)
 // but not the write; the slot convention is the one vLLM-style engines use.
 //
@@ -25,7 +25,11 @@ struct CacheWriteParams {
     int64_t num_slots;         // num_blocks * block_size
     int32_t num_tokens;
     int32_t chunks_per_token;  // Hkv * D / 8
-    float k_scale, v_scale;
+    int32_t chunks_per_head;   // D / 8
+    float k_scale, v_scale;    // per-tensor scales, used when k_scales is null
+    const float* k_scales;     // device scales: [1] or [Hkv] (scales_per_head)
+    const float* v_scales;
+    int32_t scales_per_head;
 };
 
 // Eight f16 values divided by `scale` in fp32 (IEEE division), rounded to
@@ -56,6 +60,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
     grid_dependents_launch();
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t total = static_cast<int64_t>(p.num_tokens) * p.chunks_per_token;
+    if (kFp8 && p.k_scales && idx == 0)
+        check_scales(p.k_scales, p.v_scales, p.scales_per_head ? p.chunks_per_token / p.chunks_per_head : 1, 0, 1);
     if (idx >= total) return;
     const int32_t tok = static_cast<int32_t>(idx / p.chunks_per_token);
     const int32_t chunk = static_cast<int32_t>(idx - static_cast<int64_t>(tok) * p.chunks_per_token);
@@ -70,8 +76,14 @@ __global__ void __launch_bounds__(256) cache_write_kernel(CacheWriteParams p) {
     // chunk c of (slot) is at chunk index slot * chunks_per_token + c in both layouts
     const int64_t dst = slot * p.chunks_per_token + chunk;
     if constexpr (kFp8) {
-        reinterpret_cast<uint2*>(p.k_cache)[dst] = quantize8_e4m3(k, p.k_scale);
-        reinterpret_cast<uint2*>(p.v_cache)[dst] = quantize8_e4m3(v, p.v_scale);
+        float ks = p.k_scale, vs = p.v_scale;
+        if (p.k_scales) {                                   // device scales of this chunk's head
+            const int head = chunk / p.chunks_per_head;
+            ks = head_scale(p.k_scales, p.scales_per_head, head);
+            vs = head_scale(p.v_scales, p.scales_per_head, head);
+        }
+        reinterpret_cast<uint2*>(p.k_cache)[dst] = quantize8_e4m3(k, ks);
+        reinterpret_cast<uint2*>(p.v_cache)[dst] = quantize8_e4m3(v, vs);
     } else {
         reinterpret_cast<uint4*>(p.k_cache)[dst] = k;
         reinterpret_cast<uint4*>(p.v_cache)[dst] = v;

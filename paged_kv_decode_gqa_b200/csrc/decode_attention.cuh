@@ -50,8 +50,11 @@ struct DecodeParams {
     int32_t max_blocks_per_seq, num_blocks, max_context_len;
     int32_t partition_tokens;     // multiple of kPageRows
     int32_t nparts;               // partitions per sequence covered by the grid
-    float logit_scale_log2;       // softmax_scale * log2(e) (* k_scale for FP8)
-    float out_scale;              // 1 (v_scale for FP8)
+    float logit_scale_log2;       // softmax_scale * log2(e) (* k_scale for FP8 with per-tensor scales)
+    float out_scale;              // 1 (v_scale for FP8 with per-tensor scales)
+    const float* k_scales;        // FP8 device scales [1] or [Hkv], or null: then for KV head g the
+    const float* v_scales;        // logit scale is logit_scale_log2 * k_scales[g], the output v_scales[g]
+    int32_t scales_per_head;
 };
 
 template <bool kFp8, int kConsumers, int kStages>
@@ -180,6 +183,12 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
 
     // ================================ consumers ================================
     const int r = lane >> 2, c = lane & 3;      // fragment row group / column pair
+    // logit and output scales of KV head g
+    const float sl = p.k_scales ? p.logit_scale_log2 * head_scale(p.k_scales, p.scales_per_head, g)
+                                : p.logit_scale_log2;
+    const float out_scale = p.v_scales ? head_scale(p.v_scales, p.scales_per_head, g) : p.out_scale;
+    if (p.k_scales && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+        check_scales(p.k_scales, p.v_scales, p.scales_per_head ? p.Hkv : 1, 0, 1);
     uint32_t qf[8][2];
     load_q_fragments<kFp8>(
         qf, r < G ? p.q + ((int64_t)b * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, c);
@@ -195,7 +204,7 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int blk = it * kConsumers + warp;
         if (blk < nblk) {
             const int valid = blk == nblk - 1 ? last_valid : kPageRows;
-            attend_page<kFp8>(st, k_tile(s, warp), v_tile(s, warp), valid, qf, p.logit_scale_log2, lane);
+            attend_page<kFp8>(st, k_tile(s, warp), v_tile(s, warp), valid, qf, sl, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(s));
@@ -242,7 +251,7 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
             acc += red_o[(w * kGroupPad + h) * kHeadDim + d] * sc;
         }
         if (nparts_b == 1) {
-            out_g[h * kHeadDim + d] = __float2half_rn(acc / lsum * p.out_scale);
+            out_g[h * kHeadDim + d] = __float2half_rn(acc / lsum * out_scale);
         } else {
             const int64_t pr = (row0 + h) * p.nparts + part;
             p.ws_o[pr * kHeadDim + d] = acc / lsum;
@@ -290,7 +299,7 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
             __syncwarp();
-            for (int q = lane; q < nparts_b; q += 32) wh[q] *= p.out_scale / sum;
+            for (int q = lane; q < nparts_b; q += 32) wh[q] *= out_scale / sum;
         }
         consumer_sync(kCT);
         for (int h = h_first; h < G; h += h_step) {
@@ -317,7 +326,7 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
                 wsum += w;
                 acc += w * __ldcg(p.ws_o + (pr0 + q) * kHeadDim + d);
             }
-            out_g[h * kHeadDim + d] = __float2half_rn(acc / wsum * p.out_scale);
+            out_g[h * kHeadDim + d] = __float2half_rn(acc / wsum * out_scale);
         }
     }
     if (threadIdx.x == 0) p.ws_count[(int64_t)b * p.Hkv + g] = 0u;   // ready for the next call

@@ -51,6 +51,9 @@ struct BalancedParams {
     int32_t overlap_previous;     // read pages/tables/lengths before waiting on the previous launch
     float logit_scale_log2;       // softmax_scale * log2(e) (* k_scale for FP8)
     float out_scale;              // 1 (v_scale for FP8)
+    const float* k_scales;        // FP8 device scales [1] or [Hkv], or null: then for KV head g the
+    const float* v_scales;        // logit scale is logit_scale_log2 * k_scales[g], the output scale
+    int32_t scales_per_head;      // v_scales[g], and the new token is quantised with them
 };
 
 constexpr int kMergeFloats = 32 * 8 + 16;     // per warp: weights of 32 items x 8 heads, M, L
@@ -276,6 +279,19 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     };
     uint32_t qf[8][2];
     load_q_fragments<kFp8>(qf, q_row(b, g), c);
+    // scales of the current segment's KV head (device scales are read after the wait)
+    float sl = p.logit_scale_log2, out_scale = p.out_scale, k_quant = p.k_scale, v_quant = p.v_scale;
+    auto set_head_scales = [&](int gg) {
+        if (p.k_scales) {
+            k_quant = head_scale(p.k_scales, p.scales_per_head, gg);
+            v_quant = head_scale(p.v_scales, p.scales_per_head, gg);
+            sl = p.logit_scale_log2 * k_quant;
+            out_scale = v_quant;
+        }
+    };
+    set_head_scales(g);
+    if (p.k_scales && blockIdx.x == 0 && warp == 0)
+        check_scales(p.k_scales, p.v_scales, p.scales_per_head ? Hkv : 1, lane, 32);
     WarpState st;
     st.reset();
 
@@ -308,7 +324,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     auto finish_piece = [&](int j_last) {
         st.reduce_l();
         if (piece_j0 == 0 && j_last == nb - 1) {          // the whole segment: write it
-            write_out(st.o, p.out_scale / st.l0, p.out_scale / st.l1);
+            write_out(st.o, out_scale / st.l0, out_scale / st.l1);
             return;
         }
         // The segment's pieces belong to workers k_first..k_last, one each. They
@@ -414,7 +430,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (lane == 0) *cnt = 0u;                          // ready for the next call
             const int n_next = (n_items + 31) / 32;
             if (n_next == 1) {
-                write_out(acc, p.out_scale, p.out_scale);
+                write_out(acc, out_scale, out_scale);
                 return;
             }
 #pragma unroll
@@ -442,7 +458,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         const bool in_pool = pb >= 0 && pb < p.num_blocks;
         const int64_t dst = (((int64_t)pb * kPageRows + row) * Hkv + g) * kHeadDim + 4 * lane;
         if constexpr (kFp8) {
-            const uint32_t kq = quantize4_e4m3(kh, p.k_scale), vq = quantize4_e4m3(vh, p.v_scale);
+            const uint32_t kq = quantize4_e4m3(kh, k_quant), vq = quantize4_e4m3(vh, v_quant);
             const uint32_t off = row * 128 + ((((lane >> 2) ^ (row & 7))) << 4) + (lane & 3) * 4;
             asm volatile("st.shared.u32 [%0], %1;" :: "r"(k_tile(s) + off), "r"(kq) : "memory");
             asm volatile("st.shared.u32 [%0], %1;" :: "r"(v_tile(s) + off), "r"(vq) : "memory");
@@ -465,7 +481,6 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         __syncwarp();
     };
 
-    const float sl = p.logit_scale_log2;
     for (int t = 0; t < n; ++t) {
         const int s = t % kStages;
         if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (t / kStages) & 1))) return;
@@ -507,6 +522,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
                     nb = units_of(b);
                 }
                 load_q_fragments<kFp8>(qf, q_row(b, g), c);
+                set_head_scales(g);
             }
             piece_j0 = j;
         } else {

@@ -16,6 +16,7 @@
 #include "cache_write.cuh"
 #include "decode_attention.cuh"
 #include "decode_balanced.cuh"
+#include "fp8_scales.cuh"
 
 namespace {
 
@@ -53,6 +54,14 @@ constexpr int kBalMaxBatch = 8192;        // unit-order tables must fit in share
 constexpr int kBalMinUnits = 4;           // pages per worker at least (small batches)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// FP8 scales held on the device ([1] or [Hkv] floats); null arrays mean the
+// per-tensor scalar scales of the call.
+struct DeviceScales {
+    const float* k = nullptr;
+    const float* v = nullptr;
+    int32_t per_head = 0;
+};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -232,8 +241,8 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
                            const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
                            int32_t Hq, int32_t Hkv, int32_t max_blocks_per_seq, int32_t num_blocks,
                            int32_t max_context_len, float softmax_scale, float k_scale, float v_scale,
-                           void* workspace, size_t workspace_bytes, bool overlap_previous,
-                           cudaStream_t st) {
+                           const DeviceScales& ds, void* workspace, size_t workspace_bytes,
+                           bool overlap_previous, cudaStream_t st) {
     const BalancedLayout bl = balanced_layout((int64_t)grid * bal_warps(fp8), batch, Hkv);
     if (!workspace || workspace_bytes < bl.total) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
@@ -262,8 +271,12 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
     bp.min_units_per_worker = kBalMinUnits;
     bp.overlap_previous = overlap_previous ? 1 : 0;
     const float log2e = 1.4426950408889634f;
-    bp.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
-    bp.out_scale = fp8 ? v_scale : 1.f;
+    // per-tensor FP8 scales fold into these; device scales are applied per KV head in the kernel
+    bp.logit_scale_log2 = softmax_scale * (fp8 && !ds.k ? k_scale : 1.f) * log2e;
+    bp.out_scale = fp8 && !ds.k ? v_scale : 1.f;
+    bp.k_scales = fp8 ? ds.k : nullptr;
+    bp.v_scales = fp8 ? ds.v : nullptr;
+    bp.scales_per_head = ds.per_head;
     CUtensorMap mk, mv;
     if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, Hkv) ||
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, Hkv))
@@ -322,6 +335,165 @@ pkv_status check_attention_args(const void* out, const void* q, const void* k_ca
     return PKV_OK;
 }
 
+
+// ---------------------------------------------------------------- the calls
+// Bodies of the entry points, with FP8 scales either per tensor (host
+// scalars) or on the device (DeviceScales).
+
+pkv_status cache_write_impl(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                                const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t num_blocks, int32_t block_size,
+                                int32_t kv_dtype, float k_scale, float v_scale, const DeviceScales& ds,
+                            void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (head_dim % 8 != 0) return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+        return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    pkv::CacheWriteParams prm;
+    prm.k_new = static_cast<const uint4*>(k_new);
+    prm.v_new = static_cast<const uint4*>(v_new);
+    prm.k_cache = k_cache;
+    prm.v_cache = v_cache;
+    prm.slot_mapping = slot_mapping;
+    prm.num_slots = (int64_t)num_blocks * block_size;
+    prm.num_tokens = num_tokens;
+    prm.chunks_per_token = num_kv_heads * (head_dim / 8);
+    prm.chunks_per_head = head_dim / 8;
+    prm.k_scale = k_scale;
+    prm.v_scale = v_scale;
+    prm.k_scales = fp8 ? ds.k : nullptr;
+    prm.v_scales = fp8 ? ds.v : nullptr;
+    prm.scales_per_head = ds.per_head;
+    const int64_t total = (int64_t)num_tokens * prm.chunks_per_token;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        fp8 ? launch_pdl(pkv::cache_write_kernel<true>, dim3((unsigned)blocks), dim3(threads), 0, st, prm)
+            : launch_pdl(pkv::cache_write_kernel<false>, dim3((unsigned)blocks), dim3(threads), 0, st, prm);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status attention_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* context_lens,
+                                      int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                                      int32_t num_blocks, int32_t max_context_len, float softmax_scale,
+                                      int32_t kv_dtype, float k_scale, float v_scale, const DeviceScales& ds,
+                                      int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+    {
+        const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                                  num_q_heads, num_kv_heads, head_dim, block_size,
+                                                  max_blocks_per_seq, num_blocks, max_context_len,
+                                                  softmax_scale, kv_dtype, k_scale, v_scale,
+                                                  partition_tokens);
+        if (v != PKV_OK || batch == 0) return v;
+    }
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    const int G = num_q_heads / num_kv_heads;
+
+    const float log2e = 1.4426950408889634f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (partition_tokens == PKV_PARTITION_AUTO) {
+        const int grid = !use_balanced(batch, num_kv_heads, max_blocks_per_seq) ? 0
+                         : fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+        if (grid > 0) {
+            return launch_balanced(fp8, grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
+                                   context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
+                                   num_blocks, max_context_len, softmax_scale, k_scale, v_scale, ds,
+                                   workspace, workspace_bytes, false, st);
+        }
+        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
+                                                              kPageRows, 0);
+    }
+
+    // plan: a partition covering the longest context is a single pass
+    int32_t P = partition_tokens;
+    if (P == 0 || P >= max_context_len) P = std::max(max_context_len, 1);
+    P = (P + kPageRows - 1) / kPageRows * kPageRows;
+    const int nparts = std::max(1, (max_context_len + P - 1) / P);
+
+    pkv::DecodeParams prm{};
+    prm.out = static_cast<__half*>(out);
+    prm.q = static_cast<const __half*>(q);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    if (nparts > 1) {
+        const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, num_kv_heads, nparts);
+        if (!workspace || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        prm.ws_o = reinterpret_cast<float*>(ws + wl.o);
+        prm.ws_m = reinterpret_cast<float*>(ws + wl.m);
+        prm.ws_l = reinterpret_cast<float*>(ws + wl.l);
+        prm.ws_count = reinterpret_cast<unsigned int*>(ws + wl.count);
+    }
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.G = G;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition_tokens = P;
+    prm.nparts = nparts;
+    prm.logit_scale_log2 = softmax_scale * (fp8 && !ds.k ? k_scale : 1.f) * log2e;
+    prm.out_scale = fp8 && !ds.k ? v_scale : 1.f;
+    prm.k_scales = fp8 ? ds.k : nullptr;
+    prm.v_scales = fp8 ? ds.v : nullptr;
+    prm.scales_per_head = ds.per_head;
+
+    CUtensorMap mk, mv;
+    if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
+        !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
+        return PKV_ERR_CUDA;
+    return fp8 ? launch_decode<true, kStagesFp8>(prm, mk, mv, batch, num_kv_heads, st)
+               : launch_decode<false, kStagesF16>(prm, mk, mv, batch, num_kv_heads, st);
+}
+
+pkv_status step_impl(void* out, const void* q, const void* k_new, const void* v_new,
+                                 void* k_cache, void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_context_len,
+                                 float softmax_scale, int32_t kv_dtype, float k_scale, float v_scale,
+                                 const DeviceScales& ds, void* workspace, size_t workspace_bytes,
+                                 uint32_t flags, void* stream) {
+    if (flags & ~PKV_STEP_OVERLAP_PREVIOUS) return PKV_ERR_INVALID_ARG;
+    const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                              num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                                              kv_dtype, k_scale, v_scale, PKV_PARTITION_AUTO);
+    if (v != PKV_OK || batch == 0) return v;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_INVALID_ARG;
+    if (!use_balanced(batch, num_kv_heads, max_blocks_per_seq)) return PKV_ERR_UNSUPPORTED;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+    if (grid <= 0) return PKV_ERR_UNSUPPORTED;
+    return launch_balanced(fp8, grid, k_new, v_new, out, q, k_cache, v_cache, block_tables, context_lens,
+                           batch, num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks,
+                           max_context_len, softmax_scale, k_scale, v_scale, ds, workspace, workspace_bytes,
+                           (flags & PKV_STEP_OVERLAP_PREVIOUS) != 0, static_cast<cudaStream_t>(stream));
+}
+
+// Validates a device-scale pair (a per-head set needs num_kv_heads entries).
+pkv_status check_device_scales(const float* k_scales, const float* v_scales, int32_t per_head) {
+    if (!k_scales || !v_scales) return PKV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k_scales) & 3u) || (reinterpret_cast<uintptr_t>(v_scales) & 3u))
+        return PKV_ERR_INVALID_ARG;
+    if (per_head != 0 && per_head != 1) return PKV_ERR_INVALID_ARG;
+    return PKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -351,38 +523,61 @@ pkv_status paged_kv_cache_write(const void* k_new, const void* v_new, void* k_ca
                                 const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
                                 int32_t head_dim, int32_t num_blocks, int32_t block_size,
                                 int32_t kv_dtype, float k_scale, float v_scale, void* stream) {
-    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
-        return PKV_ERR_INVALID_ARG;
-    if (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
-    if (head_dim % 8 != 0) return PKV_ERR_UNSUPPORTED;
-    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
-    if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
-        return PKV_ERR_INVALID_ARG;
-    if (num_tokens == 0) return PKV_OK;
-    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
-    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
-        return PKV_ERR_INVALID_ARG;
-    pkv::CacheWriteParams prm;
-    prm.k_new = static_cast<const uint4*>(k_new);
-    prm.v_new = static_cast<const uint4*>(v_new);
-    prm.k_cache = k_cache;
-    prm.v_cache = v_cache;
-    prm.slot_mapping = slot_mapping;
-    prm.num_slots = (int64_t)num_blocks * block_size;
-    prm.num_tokens = num_tokens;
-    prm.chunks_per_token = num_kv_heads * (head_dim / 8);
-    prm.k_scale = k_scale;
-    prm.v_scale = v_scale;
-    const int64_t total = (int64_t)num_tokens * prm.chunks_per_token;
-    const int threads = 256;
-    const int64_t blocks = (total + threads - 1) / threads;
-    if (blocks > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+    return cache_write_impl(k_new, v_new, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                            num_blocks, block_size, kv_dtype, k_scale, v_scale, DeviceScales{}, stream);
+}
+
+pkv_status paged_kv_fp8_scales(const void* x, int64_t rows, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t scales_per_head, float* scales, void* stream) {
+    if (rows < 0 || num_kv_heads <= 0 || head_dim <= 0 || !scales) return PKV_ERR_INVALID_ARG;
+    if (scales_per_head != 0 && scales_per_head != 1) return PKV_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(scales) & 3u) return PKV_ERR_INVALID_ARG;
+    if (head_dim % 8 != 0 || (scales_per_head && num_kv_heads > 1024)) return PKV_ERR_UNSUPPORTED;
+    if (rows > 0 && (!x || !aligned16(x))) return PKV_ERR_INVALID_ARG;
+    const int n = scales_per_head ? num_kv_heads : 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const cudaError_t e =
-        fp8 ? launch_pdl(pkv::cache_write_kernel<true>, dim3((unsigned)blocks), dim3(threads), 0, st, prm)
-            : launch_pdl(pkv::cache_write_kernel<false>, dim3((unsigned)blocks), dim3(threads), 0, st, prm);
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    // the running maxima live in `scales` (as fp32 bit patterns) until the conversion
+    if (cudaMemsetAsync(scales, 0, sizeof(float) * n, st) != cudaSuccess) return PKV_ERR_CUDA;
+    if (rows > 0) {
+        pkv::AmaxParams ap;
+        ap.x = static_cast<const uint4*>(x);
+        ap.chunks_per_head = head_dim / 8;
+        ap.chunks = rows * num_kv_heads * (int64_t)ap.chunks_per_head;
+        ap.Hkv = num_kv_heads;
+        ap.per_head = scales_per_head;
+        ap.amax_bits = reinterpret_cast<unsigned int*>(scales);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        constexpr int kThreads = 256;
+        int64_t blocks = std::min<int64_t>((ap.chunks + kThreads - 1) / kThreads, 8 * (int64_t)sms);
+        // a grid stride that is a multiple of one row's chunks keeps each thread on one head
+        const int64_t row_chunks = (int64_t)num_kv_heads * ap.chunks_per_head;
+        if (scales_per_head && blocks * kThreads >= row_chunks) {
+            int64_t unit = row_chunks;                       // threads per whole number of rows
+            while (unit % kThreads) unit += row_chunks;
+            const int64_t unit_blocks = unit / kThreads;
+            if (unit_blocks <= blocks) blocks = blocks / unit_blocks * unit_blocks;
+        }
+        if (launch_pdl(pkv::amax_kernel, dim3((unsigned)blocks), dim3(kThreads), sizeof(unsigned int) * n, st,
+                       ap) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
+    return launch_pdl(pkv::scales_from_amax_kernel, dim3(1), dim3(256), 0, st, scales, n) == cudaSuccess
+               ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status paged_kv_cache_write_fp8_scaled(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                                           const int64_t* slot_mapping, int32_t num_tokens,
+                                           int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                           int32_t block_size, const float* k_scales, const float* v_scales,
+                                           int32_t scales_per_head, void* stream) {
+    const pkv_status v = check_device_scales(k_scales, v_scales, scales_per_head);
+    if (v != PKV_OK) return v;
+    return cache_write_impl(k_new, v_new, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                            num_blocks, block_size, PKV_KV_FP8_E4M3, 1.f, 1.f,
+                            DeviceScales{k_scales, v_scales, scales_per_head}, stream);
 }
 
 size_t paged_gqa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
@@ -441,70 +636,24 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q, const void* k_ca
                                       int32_t kv_dtype, float k_scale, float v_scale,
                                       int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                       void* stream) {
-    {
-        const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
-                                                  num_q_heads, num_kv_heads, head_dim, block_size,
-                                                  max_blocks_per_seq, num_blocks, max_context_len,
-                                                  softmax_scale, kv_dtype, k_scale, v_scale,
-                                                  partition_tokens);
-        if (v != PKV_OK || batch == 0) return v;
-    }
-    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
-    const int G = num_q_heads / num_kv_heads;
+    return attention_impl(out, q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                          kv_dtype, k_scale, v_scale, DeviceScales{}, partition_tokens, workspace,
+                          workspace_bytes, stream);
+}
 
-    const float log2e = 1.4426950408889634f;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (partition_tokens == PKV_PARTITION_AUTO) {
-        const int grid = !use_balanced(batch, num_kv_heads, max_blocks_per_seq) ? 0
-                         : fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
-        if (grid > 0) {
-            return launch_balanced(fp8, grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
-                                   context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
-                                   num_blocks, max_context_len, softmax_scale, k_scale, v_scale,
-                                   workspace, workspace_bytes, false, st);
-        }
-        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
-                                                              kPageRows, 0);
-    }
-
-    // plan: a partition covering the longest context is a single pass
-    int32_t P = partition_tokens;
-    if (P == 0 || P >= max_context_len) P = std::max(max_context_len, 1);
-    P = (P + kPageRows - 1) / kPageRows * kPageRows;
-    const int nparts = std::max(1, (max_context_len + P - 1) / P);
-
-    pkv::DecodeParams prm{};
-    prm.out = static_cast<__half*>(out);
-    prm.q = static_cast<const __half*>(q);
-    prm.block_tables = block_tables;
-    prm.context_lens = context_lens;
-    if (nparts > 1) {
-        const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, num_kv_heads, nparts);
-        if (!workspace || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
-        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
-        uint8_t* ws = static_cast<uint8_t*>(workspace);
-        prm.ws_o = reinterpret_cast<float*>(ws + wl.o);
-        prm.ws_m = reinterpret_cast<float*>(ws + wl.m);
-        prm.ws_l = reinterpret_cast<float*>(ws + wl.l);
-        prm.ws_count = reinterpret_cast<unsigned int*>(ws + wl.count);
-    }
-    prm.Hq = num_q_heads;
-    prm.Hkv = num_kv_heads;
-    prm.G = G;
-    prm.max_blocks_per_seq = max_blocks_per_seq;
-    prm.num_blocks = num_blocks;
-    prm.max_context_len = max_context_len;
-    prm.partition_tokens = P;
-    prm.nparts = nparts;
-    prm.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * log2e;
-    prm.out_scale = fp8 ? v_scale : 1.f;
-
-    CUtensorMap mk, mv;
-    if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
-        !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
-        return PKV_ERR_CUDA;
-    return fp8 ? launch_decode<true, kStagesFp8>(prm, mk, mv, batch, num_kv_heads, st)
-               : launch_decode<false, kStagesF16>(prm, mk, mv, batch, num_kv_heads, st);
+pkv_status paged_gqa_decode_attention_fp8_scaled(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_context_len,
+    float softmax_scale, const float* k_scales, const float* v_scales, int32_t scales_per_head,
+    int32_t partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+    const pkv_status v = check_device_scales(k_scales, v_scales, scales_per_head);
+    if (v != PKV_OK) return v;
+    return attention_impl(out, q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                          PKV_KV_FP8_E4M3, 1.f, 1.f, DeviceScales{k_scales, v_scales, scales_per_head},
+                          partition_tokens, workspace, workspace_bytes, stream);
 }
 
 pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
@@ -514,21 +663,24 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
                                  int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_context_len,
                                  float softmax_scale, int32_t kv_dtype, float k_scale, float v_scale,
                                  void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
-    if (flags & ~PKV_STEP_OVERLAP_PREVIOUS) return PKV_ERR_INVALID_ARG;
-    const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
-                                              num_q_heads, num_kv_heads, head_dim, block_size,
-                                              max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
-                                              kv_dtype, k_scale, v_scale, PKV_PARTITION_AUTO);
-    if (v != PKV_OK || batch == 0) return v;
-    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_INVALID_ARG;
-    if (!use_balanced(batch, num_kv_heads, max_blocks_per_seq)) return PKV_ERR_UNSUPPORTED;
-    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
-    const int grid = fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
-    if (grid <= 0) return PKV_ERR_UNSUPPORTED;
-    return launch_balanced(fp8, grid, k_new, v_new, out, q, k_cache, v_cache, block_tables, context_lens,
-                           batch, num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks,
-                           max_context_len, softmax_scale, k_scale, v_scale, workspace, workspace_bytes,
-                           (flags & PKV_STEP_OVERLAP_PREVIOUS) != 0, static_cast<cudaStream_t>(stream));
+    return step_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads,
+                     num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                     softmax_scale, kv_dtype, k_scale, v_scale, DeviceScales{}, workspace, workspace_bytes,
+                     flags, stream);
+}
+
+pkv_status paged_gqa_decode_step_fp8_scaled(
+    void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+    int32_t max_context_len, float softmax_scale, const float* k_scales, const float* v_scales,
+    int32_t scales_per_head, void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
+    const pkv_status v = check_device_scales(k_scales, v_scales, scales_per_head);
+    if (v != PKV_OK) return v;
+    return step_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads,
+                     num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                     softmax_scale, PKV_KV_FP8_E4M3, 1.f, 1.f, DeviceScales{k_scales, v_scales, scales_per_head},
+                     workspace, workspace_bytes, flags, stream);
 }
 
 }  // extern "C"

@@ -110,6 +110,32 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 16-byte global load of data read once (no L1 allocation).
+__device__ __forceinline__ uint4 ld_stream_16(const uint4* src) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(src));
+    return v;
+}
+
+// ---------------------------------------------------------- FP8 scales
+// Scale of KV head g from a device array of one element (per tensor) or one
+// per KV head.
+__device__ __forceinline__ float head_scale(const float* scales, int32_t per_head, int g) {
+    return __ldg(scales + (per_head ? g : 0));
+}
+
+// Flags device-side scales that are not positive and finite (the calling
+// threads check elements t0, t0 + nt, ... of both arrays).
+__device__ __forceinline__ void check_scales(const float* k_scales, const float* v_scales, int n, int t0,
+                                             int nt) {
+    for (int i = t0; i < n; i += nt) {
+        const float a = __ldg(k_scales + i), b = __ldg(v_scales + i);
+        if (!(a > 0.f && a <= 3.402823466e38f) || !(b > 0.f && b <= 3.402823466e38f))
+            flag_error(PKV_DEVERR_SCALE);
+    }
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

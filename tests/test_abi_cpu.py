@@ -106,6 +106,57 @@ def test_cache_write_rejects_bad_arguments_on_host(kw, status):
     assert rc == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=0), pkv.PKV_ERR_INVALID_ARG),                 # device scales missing
+    (dict(ks=A + 2), pkv.PKV_ERR_INVALID_ARG),             # misaligned float array
+    (dict(per_head=2), pkv.PKV_ERR_INVALID_ARG),
+    (dict(q=0), pkv.PKV_ERR_INVALID_ARG),                  # the attention checks still apply
+    (dict(Hq=20), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(B=0), pkv.PKV_OK),
+])
+def test_fp8_scaled_attention_rejects_bad_arguments_on_host(kw, status):
+    a = dict(out=A, q=A, k=A, v=A, bt=A, cl=A, B=2, Hq=12, Hkv=2, D=128, bs=16, mb=4, NB=64,
+             maxlen=40, scale=0.088, ks=A, vs=A, per_head=1, P=0, ws=0, wsb=0)
+    a.update(kw)
+    rc = pkv.load_library().paged_gqa_decode_attention_fp8_scaled(
+        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"],
+        a["mb"], a["NB"], a["maxlen"], a["scale"], a["ks"], a["vs"], a["per_head"], a["P"], a["ws"],
+        a["wsb"], None)
+    assert rc == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(vs=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(per_head=-1), pkv.PKV_ERR_INVALID_ARG),
+    (dict(D=12), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(T=0), pkv.PKV_OK),
+])
+def test_fp8_scaled_cache_write_rejects_bad_arguments_on_host(kw, status):
+    a = dict(k_new=A, v_new=A, kc=A, vc=A, slots=A, T=4, Hkv=2, D=128, NB=64, bs=16, ks=A, vs=A, per_head=0)
+    a.update(kw)
+    rc = pkv.load_library().paged_kv_cache_write_fp8_scaled(
+        a["k_new"], a["v_new"], a["kc"], a["vc"], a["slots"], a["T"], a["Hkv"], a["D"], a["NB"], a["bs"],
+        a["ks"], a["vs"], a["per_head"], None)
+    assert rc == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(scales=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(x=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(x=A + 8), pkv.PKV_ERR_INVALID_ARG),              # chunks are 16-byte loads
+    (dict(D=12), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(Hkv=2000), pkv.PKV_ERR_UNSUPPORTED),             # per-head maxima live in shared memory
+    (dict(rows=-1), pkv.PKV_ERR_INVALID_ARG),
+    (dict(per_head=3), pkv.PKV_ERR_INVALID_ARG),
+])
+def test_fp8_scales_rejects_bad_arguments_on_host(kw, status):
+    a = dict(x=A, rows=64, Hkv=2, D=128, per_head=1, scales=A)
+    a.update(kw)
+    rc = pkv.load_library().paged_kv_fp8_scales(a["x"], a["rows"], a["Hkv"], a["D"], a["per_head"],
+                                                a["scales"], None)
+    assert rc == status
+
+
 def test_pages_head_counts_give_the_6x_kv_read_cut():
     """The GQA read saving the page quotes is Hq/Hkv under the byte model bench.py reports."""
     import json
