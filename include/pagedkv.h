@@ -78,7 +78,7 @@ typedef enum {
 
 typedef enum {
     PKV_KV_F16 = 0,            /* float16 cache */
-    PKV_KV_FP8_E4M3 = 1        /* uint8 OCP E4M3 cache with per-tensor scales */
+    PKV_KV_FP8_E4M3 = 1        /* uint8 OCP E4M3 cache, per-tensor or per-KV-head scales */
 } pkv_kv_dtype;
 
 /* partition_tokens value that lets the library plan the split-KV work: the

@@ -32,7 +32,7 @@ constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 // thread). Measured best on the benchmark workloads with two-page softmax
 // steps: f16 6 workers x 3 slots (144 KiB of ring; 8 x 3 took 17% longer on
 // the 1.5B-shaped step and 25% on the skewed one, 7B-shaped steps were within
-// 2% for 5..8 workers), FP8 8 workers x 4 slots (64 KiB; 8 x 6 and 7 x 6 were
+// 2% for 5..8 workers), FP8 8 workers x 4 slots (128 KiB; 8 x 6 and 7 x 6 were
 // slower). The macros exist for tuning builds.
 #ifndef PKV_BAL_WARPS_F16
 #define PKV_BAL_WARPS_F16 6
