@@ -9,8 +9,9 @@ compiled here with gcc into ``oracle/_build/liboracle.so``.
 What each function computes, and the readings it takes where the pages are
 silent, is stated in ``pkv_oracle.c``. Sources: "rvLLM 소개"
 (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3 (paged KV cache,
-grouped-query heads, f16 and FP8 E4M3 caches) and the vLLM talk summary
-(aitrends.kr), §용어 해설 (KV cache, PagedAttention).
+grouped-query heads, f16 and FP8 E4M3 caches), §퓨즈드 CUDA 커널 (the fused
+Add+RMSNorm+QKV step before attention) and the vLLM talk summary (aitrends.kr),
+§용어 해설 (KV cache, PagedAttention).
 
 Arrays are NumPy. binary16 data is passed as ``np.float16`` (its bits are
 read, never converted by NumPy); FP8 caches are ``np.uint8`` codes.
@@ -72,6 +73,10 @@ def _load():
         lib.oracle_absmax_f16.restype = None
         lib.oracle_fp8_scale_from_amax.argtypes = [f32]
         lib.oracle_fp8_scale_from_amax.restype = f32
+        lib.oracle_f16_from_f64.argtypes = [ctypes.c_double]
+        lib.oracle_f16_from_f64.restype = ctypes.c_uint16
+        lib.oracle_add_rmsnorm_qkv.argtypes = [P, P, P, P, P, i32, i32, i32, ctypes.c_double, P, P]
+        lib.oracle_add_rmsnorm_qkv.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -231,3 +236,42 @@ def fp8_scale_from_amax(amax):
 def fp8_scales(x, per_head: bool):
     """Scales an E4M3 cache would use for the data x [rows, Hkv, D] float16."""
     return fp8_scale_from_amax(absmax_f16(x, per_head))
+
+
+def f16_from_f64(x) -> np.ndarray:
+    """Round float64 values to binary16 codes (uint16): nearest, ties to even, overflow to inf."""
+    lib = _load()
+    x = np.asarray(x, dtype=np.float64).ravel()
+    return np.array([lib.oracle_f16_from_f64(float(v)) for v in x], dtype=np.uint16)
+
+
+def add_rmsnorm_qkv(x, residual, gamma, w_qkv, bias, eps, Hq, Hkv, D):
+    """Residual add, RMSNorm and QKV projection of one decode step, in float64.
+
+    x, residual: [T, H] float16. gamma: [H] float16. w_qkv: [(Hq + 2 Hkv) D, H]
+    float16, rows ordered query heads, key heads, value heads. bias: [N]
+    float16 or None. Returns (residual_out [T, H] float16, q [T, Hq, D],
+    k [T, Hkv, D], v [T, Hkv, D] float64).
+    """
+    x = _c(x, np.float16)
+    residual = _c(residual, np.float16)
+    gamma = _c(gamma, np.float16)
+    w_qkv = _c(w_qkv, np.float16)
+    T, H = x.shape
+    N = (Hq + 2 * Hkv) * D
+    if residual.shape != (T, H) or gamma.shape != (H,) or w_qkv.shape != (N, H):
+        raise ValueError("shape mismatch")
+    if bias is not None:
+        bias = _c(bias, np.float16)
+        if bias.shape != (N,):
+            raise ValueError("bias must be [N]")
+    res_out = np.empty((T, H), dtype=np.float16)
+    qkv = np.empty((T, N), dtype=np.float64)
+    rc = _load().oracle_add_rmsnorm_qkv(_ptr(x), _ptr(residual), _ptr(gamma), _ptr(w_qkv), _ptr(bias),
+                                        T, H, N, float(eps), _ptr(res_out), _ptr(qkv))
+    if rc != 0:
+        raise ValueError("bad sizes or eps")
+    q = qkv[:, :Hq * D].reshape(T, Hq, D)
+    k = qkv[:, Hq * D:(Hq + Hkv) * D].reshape(T, Hkv, D)
+    v = qkv[:, (Hq + Hkv) * D:].reshape(T, Hkv, D)
+    return res_out, q, k, v

@@ -37,6 +37,19 @@
  *      computed from data is fp32(amax) / 448 divided in fp32, amax being
  *      the largest |x| over the non-NaN elements (per head, or over the
  *      whole tensor), and 1 when that maximum is 0 (or no element counts).
+ *  Fused Add+RMSNorm+QKV ("rvLLM 소개", §퓨즈드 CUDA 커널: each layer runs
+ *  the residual add, the RMSNorm and the QKV projection as one fused kernel
+ *  whose outputs feed attention and the cache write); the page gives no
+ *  formula, so:
+ *   R9  the add is s = x + residual, rounded once to binary16 (nearest
+ *       even); s is the new residual stream and is returned;
+ *   R10 RMSNorm is y_k = s_k / sqrt(mean_k(s_k^2) + eps) * gamma_k over the
+ *       hidden size H, from the binary16 s, in float64;
+ *   R11 the projection is qkv_n = sum_k W[n][k] * y_k (+ bias_n when a bias
+ *       is given) with W [N, H] row-major and N = (Hq + 2 Hkv) * D; rows
+ *       [0, Hq D) are the query heads, the next Hkv D the key heads, the
+ *       last Hkv D the value heads, each head's D rows consecutive; no
+ *       rotary embedding is applied (the pages name none).
  *
  * Build: gcc -O2 -fopenmp -fPIC -shared -ffp-contract=off (no fast-math).
  */
@@ -341,6 +354,70 @@ int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
     free(ks);
     free(vs);
     return rc;
+}
+
+/* ------------------------------------------------ fused Add+RMSNorm+QKV */
+
+/* Round a float64 value to binary16 (R9): nearest representable value, ties
+ * to the even significand; magnitudes from 65520 (halfway between 65504 and
+ * 2^16) up become infinity; NaN gives 0x7E00. Written from the definition:
+ * in the binade [2^E, 2^(E+1)) with E >= -14 the spacing is 2^(E-10); below
+ * 2^-14 (subnormals) it is 2^-24. */
+uint16_t oracle_f16_from_f64(double x) {
+    if (isnan(x)) return 0x7E00;
+    uint16_t sign = signbit(x) ? 0x8000 : 0x0000;
+    double a = fabs(x);
+    if (a >= 65520.0) return sign | 0x7C00;
+    int E;
+    frexp(a, &E);
+    int binade = E - 1;
+    if (a == 0.0 || binade < -14) binade = -14;
+    double quantum = ldexp(1.0, binade - 10);
+    double r = quantum * rint(a / quantum);         /* a / quantum is exact */
+    if (r == 0.0) return sign;
+    int rE;
+    frexp(r, &rE);                                  /* r may have reached the next binade */
+    int rb = rE - 1;
+    int code;
+    if (rb < -14)
+        code = (int)(r / ldexp(1.0, -24));          /* subnormal: r = f * 2^-24 */
+    else
+        code = ((rb + 15) << 10) | ((int)(r / ldexp(1.0, rb - 10)) - 1024);
+    return sign | (uint16_t)code;
+}
+
+/* One decode step's residual add, RMSNorm and QKV projection (R9-R11).
+ * x, residual: [T, H] binary16; gamma: [H]; w: [N, H]; bias: [N] or NULL.
+ * Writes residual_out [T, H] (binary16 codes of s) and qkv [T, N] in
+ * float64. eps must be >= 0; returns -1 on bad sizes. */
+int oracle_add_rmsnorm_qkv(const uint16_t* x, const uint16_t* residual, const uint16_t* gamma,
+                           const uint16_t* w, const uint16_t* bias, int T, int H, int N,
+                           double eps, uint16_t* residual_out, double* qkv) {
+    if (T < 0 || H <= 0 || N <= 0 || !(eps >= 0.0)) return -1;
+#pragma omp parallel for schedule(dynamic)
+    for (int t = 0; t < T; ++t) {
+        double* y = (double*)malloc(sizeof(double) * (size_t)H);
+        double sumsq = 0.0;
+        for (int k = 0; k < H; ++k) {               /* R9: s = f16(x + residual) */
+            int64_t i = (int64_t)t * H + k;
+            double sum = oracle_f16_to_f64(x[i]) + oracle_f16_to_f64(residual[i]);   /* exact */
+            uint16_t s16 = oracle_f16_from_f64(sum);
+            residual_out[i] = s16;
+            y[k] = oracle_f16_to_f64(s16);
+            sumsq += y[k] * y[k];
+        }
+        double inv_rms = 1.0 / sqrt(sumsq / H + eps);                              /* R10 */
+        for (int k = 0; k < H; ++k) y[k] = y[k] * inv_rms * oracle_f16_to_f64(gamma[k]);
+        for (int n = 0; n < N; ++n) {               /* R11 */
+            const uint16_t* wr = w + (int64_t)n * H;
+            double acc = 0.0;
+            for (int k = 0; k < H; ++k) acc += oracle_f16_to_f64(wr[k]) * y[k];
+            if (bias) acc += oracle_f16_to_f64(bias[n]);
+            qkv[(int64_t)t * N + n] = acc;
+        }
+        free(y);
+    }
+    return 0;
 }
 
 /* Number of threads the OpenMP runtime would use for a parallel region. */

@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_qkv as qkv_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pkv_oracle.c")
 
@@ -37,6 +38,20 @@ MUTATIONS = {
                        "double r = floor(a / quantum + 0.5) * quantum;"),
     "cache_write_row": ("int64_t blk = s / block_size, row = s % block_size;",
                         "int64_t blk = s / block_size, row = (s + 1) % block_size;"),
+    # fused residual add + RMSNorm + QKV projection
+    "f16_ties_away": ("double r = quantum * rint(a / quantum);",
+                      "double r = quantum * floor(a / quantum + 0.5);"),
+    "f16_overflow_early": ("if (a >= 65520.0) return sign | 0x7C00;",
+                           "if (a > 65504.0) return sign | 0x7C00;"),
+    "residual_unrounded": ("y[k] = oracle_f16_to_f64(s16);", "y[k] = sum;"),
+    "rms_mean_off_by_one": ("double inv_rms = 1.0 / sqrt(sumsq / H + eps);",
+                            "double inv_rms = 1.0 / sqrt(sumsq / (H + 1) + eps);"),
+    "rms_eps_dropped": ("double inv_rms = 1.0 / sqrt(sumsq / H + eps);",
+                        "double inv_rms = 1.0 / sqrt(sumsq / H);"),
+    "gamma_dropped": ("y[k] = y[k] * inv_rms * oracle_f16_to_f64(gamma[k]);", "y[k] = y[k] * inv_rms;"),
+    "weight_transposed": ("acc += oracle_f16_to_f64(wr[k]) * y[k];",
+                          "acc += oracle_f16_to_f64(w[(int64_t)k * N + n]) * y[k];"),
+    "bias_dropped": ("if (bias) acc += oracle_f16_to_f64(bias[n]);", ";"),
 }
 
 PIN_TESTS = [
@@ -50,6 +65,12 @@ PIN_TESTS = [
     lambda: pins.test_worked_example_closed_form(),
     lambda: pins.test_split_merge_equals_single_pass(8),
     lambda: pins.test_head_map_contiguous_groups(),
+    lambda: qkv_pins.test_f16_rounding_ties_and_limits(),
+    lambda: qkv_pins.test_residual_add_rounds_once_to_nearest_even(),
+    lambda: qkv_pins.test_worked_example_by_hand(),
+    lambda: qkv_pins.test_constant_row_and_eps(),
+    lambda: qkv_pins.test_unit_rows_select_the_normalised_stream(),
+    lambda: qkv_pins.test_qkv_split_follows_the_row_order(),
 ]
 
 

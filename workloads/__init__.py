@@ -193,6 +193,39 @@ def _amax(x: np.ndarray) -> float:
     return float(np.abs(x.astype(np.float32)).max()) if x.size else 0.0
 
 
+# Hidden sizes of the two Qwen2.5 shapes: H = Hq * D (12 * 128 and 28 * 128).
+QKV_SHAPES = {
+    "qwen2.5-1.5b": dict(T=64, H=1536, Hq=12, Hkv=2, D=128),
+    "qwen2.5-7b": dict(T=128, H=3584, Hq=28, Hkv=4, D=128),
+}
+RMS_EPS = 1e-6
+
+
+def make_qkv_inputs(T: int, H: int, Hq: int, Hkv: int, D: int, seed: int = 0, *,
+                    bias: bool = True, outliers: bool = False) -> dict:
+    """Inputs of the fused residual add + RMSNorm + QKV projection, as NumPy arrays.
+
+    Keys: x [T,H] f16 ~ N(0,1) (the sublayer output); residual [T,H] f16 ~ N(0, 4^2)
+    (the residual stream); gamma [H] f16 ~ N(1, 0.25^2); w_qkv [(Hq+2Hkv)D, H] f16
+    ~ N(0, 1/H) (random-init weights, rows q heads | k heads | v heads); bias [N]
+    f16 ~ N(0, 0.5^2) or None. ``outliers`` plants a few large residual channels
+    (|value| up to 3e4, gamma up to 8 there), as real residual streams carry.
+    """
+    rng = np.random.default_rng(seed)
+    N = (Hq + 2 * Hkv) * D
+    x = _normal_f16(rng, (T, H))
+    residual = (rng.standard_normal((T, H), dtype=np.float32) * 4.0).astype(np.float16)
+    gamma = (1.0 + 0.25 * rng.standard_normal(H, dtype=np.float32)).astype(np.float16)
+    w = (rng.standard_normal((N, H), dtype=np.float32) / np.float32(np.sqrt(H))).astype(np.float16)
+    b = (0.5 * rng.standard_normal(N, dtype=np.float32)).astype(np.float16) if bias else None
+    if outliers and T > 0:
+        ch = rng.choice(H, size=min(4, H), replace=False)
+        residual[:, ch] = (rng.choice([-1.0, 1.0], size=(T, ch.size)) *
+                           rng.uniform(1e4, 3e4, size=(T, ch.size))).astype(np.float16)
+        gamma[ch] = np.float16(8.0)
+    return dict(x=x, residual=residual, gamma=gamma, w_qkv=w, bias=b)
+
+
 def shard_seed(seed: int, rank: int) -> int:
     """Seed of rank ``rank`` when every rank runs its own batch (weak scaling)."""
     return seed * 1000003 + rank
