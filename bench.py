@@ -231,6 +231,57 @@ def oracle_sample(w, x, max_seqs: int):
 
 
 # ---------------------------------------------------------------------- main
+def qkv_bytes(T: int, H: int, N: int, bias: bool) -> int:
+    """Algorithmic bytes of one fused add + RMSNorm + QKV launch: W once, x and residual in,
+    residual_out and q|k|v out, gamma and bias."""
+    return 2 * (N * H + 3 * T * H + T * N + H + (N if bias else 0))
+
+
+def time_qkv_projection(w, device, stream, peak, seed=0):
+    """fused_add_rmsnorm_qkv at the workload's model shape (H = Hq * D) for its batch, from a CUDA
+    graph that rotates over enough weight replicas that W is read from HBM every launch."""
+    Hq, Hkv, D, T = w.Hq, w.Hkv, w.head_dim, w.B
+    H, N = Hq * D, (Hq + 2 * Hkv) * D
+    d = W.make_qkv_inputs(T, H, Hq, Hkv, D, seed)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    x, r, g, b = t(d["x"]), t(d["residual"]), t(d["gamma"]), t(d["bias"])
+    w0 = t(d["w_qkv"])
+    R = max(2, min(64, -(-2 * L2_BYTES // (N * H * 2))))
+    ws = [w0] + [w0.clone() for _ in range(R - 1)]
+    res = torch.empty((T, H), dtype=torch.float16, device=device)
+    q = torch.empty((T, Hq, D), dtype=torch.float16, device=device)
+    kn = torch.empty((T, Hkv, D), dtype=torch.float16, device=device)
+    vn = torch.empty((T, Hkv, D), dtype=torch.float16, device=device)
+    call = lambda wi: pkv.fused_add_rmsnorm_qkv(x, r, g, wi, b, res, q, kn, vn, eps=W.RMS_EPS,
+                                                flags=pkv.PKV_STEP_OVERLAP_PREVIOUS, stream=stream)
+    with torch.cuda.stream(stream):
+        for wi in ws[:3]:
+            call(wi)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for wi in ws:
+                call(wi)
+        for _ in range(3):
+            graph.replay()
+        reps = max(1, 2000 // R)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1000 / (reps * R)
+    nbytes = qkv_bytes(T, H, N, True)
+    del graph
+    return {"what": "fused_add_rmsnorm_qkv (residual add + RMSNorm + QKV projection, q/k/v out)",
+            "T": T, "H": H, "N": N, "bias": True, "algorithmic_bytes": nbytes, "us": us,
+            "achieved": nbytes / us / 1e3, "peak": peak, "unit": "GB/s", "frac": nbytes / us / 1e3 / peak,
+            "bound": "hbm", "launches": reps * R,
+            "l2": f"{R} weight replicas rotated ({R * N * H * 2 / 2**20:.0f} MiB), graph of {R} launches, "
+                  "PKV_STEP_OVERLAP_PREVIOUS"}
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -247,6 +298,8 @@ def parse_args(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="two launches per step (cache write, then attention) instead of the fused step")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-qkv", action="store_true",
+                    help="skip timing the fused add + RMSNorm + QKV projection at the workload's shape")
     ap.add_argument("--fp8-scales", default="tensor", choices=["tensor", "per-head"],
                     help="FP8 workloads: per-tensor host scales, or per-KV-head scales computed on the "
                          "device and passed to the device-scale entry points")
@@ -534,6 +587,8 @@ def run_ours(args):
         }
         if scales_kernel:
             line["fp8_scales_kernel"] = scales_kernel
+        if not args.no_qkv:
+            line["qkv_kernel"] = time_qkv_projection(w, device, stream, peak, args.seed)
         if e2e:
             line["e2e"] = e2e
         if world == 1 and args.cpu_baseline_s > 0:

@@ -231,6 +231,58 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
                                  void* workspace, size_t workspace_bytes, uint32_t flags,
                                  void* stream);
 
+/*
+ * fused_add_rmsnorm_qkv -- the step before attention, fused: residual add,
+ * RMSNorm and the QKV projection of num_tokens decode tokens in one launch,
+ * writing q in the layout paged_gqa_decode_attention / _step take and k_new,
+ * v_new in the layout the cache write and the fused step take.
+ *
+ * "rvLLM 소개" (discuss.pytorch.kr), §퓨즈드 CUDA 커널: every layer runs the
+ * residual add, the RMSNorm and the QKV projection as one kernel (Add+RMSNorm
+ * +QKV GEMV), so the normalised activations are never written out. The page
+ * gives no formula; this library's reading, with T = num_tokens, H = hidden,
+ * D = head_dim and N = (num_q_heads + 2 num_kv_heads) * D:
+ *   residual_out[t] = f16(x[t] + residual[t])      (one rounding, nearest even)
+ *   y[t]            = s / sqrt(mean_k(s_k^2) + eps) * gamma,  s = residual_out[t]
+ *   qkv[t][n]       = sum_k w_qkv[n][k] * y[t][k] + bias[n]   (bias may be NULL)
+ * where rows [0, Hq D) of w_qkv give q[t] ([T, Hq, D]), the next Hkv D rows
+ * k_new[t] and the last Hkv D rows v_new[t] ([T, Hkv, D]), each head's D rows
+ * consecutive, as in a fused qkv_proj weight. No rotary embedding is applied
+ * (the pages name none).
+ *
+ * Arguments (device pointers, float16, row-major, 16-byte aligned):
+ *   x, residual     [T, H]       the sublayer output and the residual stream
+ *   gamma           [H]          RMSNorm weight
+ *   w_qkv           [N, H]       projection weight; bias [N] or NULL
+ *   residual_out    [T, H]       s, the new residual stream
+ *   q, k_new, v_new [T, Hq, D], [T, Hkv, D], [T, Hkv, D]
+ * No output may overlap x, residual or another output (residual_out cannot
+ * update `residual` in place: other CTAs still read it).
+ *
+ * Precision: residual_out is exact (bit-for-bit the rounded sum). q, k_new,
+ * v_new are f16 (nearest even) of an fp32-accumulated dot product whose
+ * activation operand is f16(s * gamma * 2^-e_t), e_t a per-token power of
+ * two chosen so that no operand overflows; the 1/RMS factor is applied in
+ * fp32 after the sum. The error is within 2^-10 * sum_k |w[n][k] y[t][k]|
+ * plus the output rounding.
+ *
+ * Supported: H a multiple of 64 and at most 10240, D a multiple of 8,
+ * N <= 2^24, T <= 4194240; others return PKV_ERR_UNSUPPORTED. eps must be
+ * finite and >= 0. T == 0 is a no-op (the per-token pointers may then be
+ * NULL; gamma and w_qkv may not).
+ *
+ * flags: 0, or PKV_STEP_OVERLAP_PREVIOUS. The kernel is launched with
+ * programmatic dependent launch. With the flag it requests its first weight
+ * tiles before waiting for the previous launch in `stream`: the caller
+ * promises that launch does not write w_qkv.
+ */
+pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void* gamma,
+                                 const void* w_qkv, const void* bias, void* residual_out,
+                                 void* q, void* k_new, void* v_new,
+                                 int32_t num_tokens, int32_t hidden, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, float eps,
+                                 uint32_t flags, void* stream);
+
 /* Static text for a status code. Never NULL. */
 const char* pkv_status_string(pkv_status status);
 

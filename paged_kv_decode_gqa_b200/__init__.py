@@ -48,6 +48,8 @@ _SIGNATURES = {
     "paged_gqa_decode_step_fp8_scaled": (
         [_P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _P, _P, _i32,
          _P, _sz, ctypes.c_uint32, _P], ctypes.c_int),
+    "fused_add_rmsnorm_qkv": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _f32,
+                               ctypes.c_uint32, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -335,3 +337,29 @@ def paged_gqa_decode_step_fp8_scaled(out, q, k_new, v_new, k_cache, v_cache, blo
         _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
         float(softmax_scale), _ptr(k_scales), _ptr(v_scales), per_head, _ptr(workspace), ws_bytes,
         int(flags), _stream(stream)), "paged_gqa_decode_step_fp8_scaled")
+
+
+def fused_add_rmsnorm_qkv(x, residual, gamma, w_qkv, bias, residual_out, q, k_new, v_new, *, eps=1e-6,
+                          flags=0, stream=None) -> None:
+    """residual_out = x + residual (f16); q, k_new, v_new = the QKV projection of its RMSNorm.
+
+    x, residual, residual_out [T, H]; gamma [H]; w_qkv [(Hq + 2 Hkv) D, H] (rows q heads | k | v);
+    bias [N] or None; q [T, Hq, D]; k_new, v_new [T, Hkv, D]; all float16.
+    """
+    for n, t in (("x", x), ("residual", residual), ("gamma", gamma), ("w_qkv", w_qkv),
+                 ("residual_out", residual_out), ("q", q), ("k_new", k_new), ("v_new", v_new)):
+        _dense(n, t, "float16")
+    if bias is not None:
+        _dense("bias", bias, "float16")
+    T, H = x.shape
+    _, Hq, D = q.shape
+    Hkv = k_new.shape[1]
+    if (residual.shape != (T, H) or residual_out.shape != (T, H) or gamma.shape != (H,)
+            or q.shape != (T, Hq, D) or k_new.shape != (T, Hkv, D) or v_new.shape != (T, Hkv, D)
+            or w_qkv.shape != ((Hq + 2 * Hkv) * D, H)
+            or (bias is not None and bias.shape != ((Hq + 2 * Hkv) * D,))):
+        raise ValueError("shape mismatch")
+    _check(load_library().fused_add_rmsnorm_qkv(
+        _ptr(x), _ptr(residual), _ptr(gamma), _ptr(w_qkv), _ptr(bias), _ptr(residual_out), _ptr(q),
+        _ptr(k_new), _ptr(v_new), T, H, Hq, Hkv, D, float(eps), int(flags), _stream(stream)),
+        "fused_add_rmsnorm_qkv")

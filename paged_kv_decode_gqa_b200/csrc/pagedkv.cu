@@ -17,6 +17,7 @@
 #include "decode_attention.cuh"
 #include "decode_balanced.cuh"
 #include "fp8_scales.cuh"
+#include "qkv_proj.cuh"
 
 namespace {
 
@@ -494,6 +495,139 @@ pkv_status check_device_scales(const float* k_scales, const float* v_scales, int
     return PKV_OK;
 }
 
+// ------------------------------------------------ fused add + RMSNorm + QKV
+// One CTA shape per weight-tile height: 128 rows with a 4-slot ring (16 KiB
+// slots), 256 rows with a 3-slot ring (32 KiB slots); the rest of the shared
+// memory holds the activation slice.
+constexpr int kQkvStages1 = 4;
+constexpr int kQkvStages2 = 3;
+constexpr int kQkvMaxSplit = 8;                 // portable cluster size
+template <int kMT>
+using QkvShapeT = pkv::QkvShape<kMT, kMT == 1 ? kQkvStages1 : kQkvStages2>;
+template <int kMT>
+auto qkv_kernel() { return pkv::add_rmsnorm_qkv_kernel<kMT, kMT == 1 ? kQkvStages1 : kQkvStages2>; }
+
+// W [N, H] f16 as a 2-D TMA tensor (k, feature) with [rows x 64] boxes,
+// 128-byte swizzled; rows past N read as zeros.
+bool make_w_map(CUtensorMap* map, const void* w, int H, int N, int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)H, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)H * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)rows};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct QkvPlan {
+    int mt = 0, split = 0, slab_blocks = 0, ftiles = 0, ttiles = 0;
+    size_t smem = 0;
+    int64_t cost = 0;
+};
+
+template <int kMT>
+cudaLaunchConfig_t qkv_config(const QkvPlan& pl, cudaStream_t st, cudaLaunchAttribute (&attr)[2]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(pl.ftiles * pl.split), (unsigned)pl.ttiles);
+    cfg.blockDim = dim3(QkvShapeT<kMT>::kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)pl.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cfg;
+}
+
+// The plan for one tile height: as many slices of H per tile as fill the
+// SMs in one wave, at least as many as the activation slice needs, and one
+// that the device can schedule as a cluster. Its cost is the W bytes a CTA
+// streams times the waves. False if no split fits.
+template <int kMT>
+bool qkv_candidate(int T, int H, int N, int sms, QkvPlan* out) {
+    using S = QkvShapeT<kMT>;
+    static unsigned long long done = 0;
+    auto kernel = qkv_kernel<kMT>();
+    if (ensure_smem(kernel, (int)S::smem_bytes(S::kMaxSlabBlocks), &done) != cudaSuccess) return false;
+    const int kb = H / 64;
+    QkvPlan pl;
+    pl.mt = kMT;
+    pl.ftiles = (N + S::kFT - 1) / S::kFT;
+    pl.ttiles = (T + S::kTT - 1) / S::kTT;
+    const int tiles = pl.ftiles * pl.ttiles;
+    const int split_min = (kb + S::kMaxSlabBlocks - 1) / S::kMaxSlabBlocks;
+    const int split_max = std::min(kQkvMaxSplit, kb);
+    if (split_min > split_max) return false;
+    for (int split = std::max(split_min, std::min(split_max, sms / std::max(tiles, 1))); split >= split_min;
+         --split) {
+        pl.split = split;
+        pl.slab_blocks = (kb + split - 1) / split;
+        pl.smem = S::smem_bytes(pl.slab_blocks);
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = qkv_config<kMT>(pl, nullptr, attr);
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        if (clusters < 1) continue;
+        const int64_t ctas = (int64_t)tiles * split;
+        const int64_t slots = std::max<int64_t>(1, std::min<int64_t>((int64_t)clusters * split, sms));
+        pl.cost = (ctas + slots - 1) / slots * S::kFT * pl.slab_blocks;
+        *out = pl;
+        return true;
+    }
+    return false;
+}
+
+bool qkv_plan(int T, int H, int N, QkvPlan* out) {
+    struct Entry {
+        int dev, T, H, N;
+        QkvPlan plan;
+    };
+    constexpr int kSlots = 8;
+    thread_local Entry cache[kSlots];
+    thread_local int used = 0, next = 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return false;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].dev == dev && cache[i].T == T && cache[i].H == H && cache[i].N == N) {
+            *out = cache[i].plan;
+            return true;
+        }
+    QkvPlan a, b;
+    const bool ha = qkv_candidate<1>(T, H, N, sms, &a);
+    const bool hb = qkv_candidate<2>(T, H, N, sms, &b);
+    if (!ha && !hb) return false;
+    *out = (ha && (!hb || a.cost <= b.cost)) ? a : b;
+    cache[next] = Entry{dev, T, H, N, *out};
+    next = (next + 1) % kSlots;
+    used = std::min(used + 1, kSlots);
+    return true;
+}
+
+template <int kMT>
+pkv_status launch_qkv(const QkvPlan& pl, const pkv::QkvParams& prm, const void* w, cudaStream_t st) {
+    CUtensorMap map;
+    if (!make_w_map(&map, w, prm.H, prm.N, QkvShapeT<kMT>::kFT)) return PKV_ERR_CUDA;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = qkv_config<kMT>(pl, st, attr);
+    return cudaLaunchKernelEx(&cfg, qkv_kernel<kMT>(), map, prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+bool ranges_overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na > 0 && nb > 0 && x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
+}
+
 }  // namespace
 
 extern "C" {
@@ -681,6 +815,62 @@ pkv_status paged_gqa_decode_step_fp8_scaled(
                      num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
                      softmax_scale, PKV_KV_FP8_E4M3, 1.f, 1.f, DeviceScales{k_scales, v_scales, scales_per_head},
                      workspace, workspace_bytes, flags, stream);
+}
+
+pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void* gamma, const void* w_qkv,
+                                 const void* bias, void* residual_out, void* q, void* k_new, void* v_new,
+                                 int32_t num_tokens, int32_t hidden, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, float eps, uint32_t flags, void* stream) {
+    if (flags & ~PKV_STEP_OVERLAP_PREVIOUS) return PKV_ERR_INVALID_ARG;
+    if (num_tokens < 0 || hidden <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (!(eps >= 0.f && eps <= 3.402823466e38f)) return PKV_ERR_INVALID_ARG;
+    // the per-token buffers are empty (possibly null) when there are no tokens
+    const void* weights[] = {gamma, w_qkv};
+    const void* per_token[] = {x, residual, residual_out, q, k_new, v_new};
+    for (const void* ptr : weights)
+        if (!ptr || !aligned16(ptr)) return PKV_ERR_INVALID_ARG;
+    for (const void* ptr : per_token)
+        if ((num_tokens > 0 && !ptr) || !aligned16(ptr)) return PKV_ERR_INVALID_ARG;
+    if (bias && !aligned16(bias)) return PKV_ERR_INVALID_ARG;
+    const int64_t N = ((int64_t)num_q_heads + 2 * (int64_t)num_kv_heads) * head_dim;
+    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxSplit * 64 * QkvShapeT<1>::kMaxSlabBlocks ||
+        N > (1 << 24) || num_tokens > 65535 * 64)
+        return PKV_ERR_UNSUPPORTED;
+    const int64_t T = num_tokens;
+    const int64_t act = T * hidden * 2, qb = T * num_q_heads * head_dim * 2, kvb = T * num_kv_heads * head_dim * 2;
+    const void* outs[] = {residual_out, q, k_new, v_new};
+    const int64_t out_bytes[] = {act, qb, kvb, kvb};
+    for (int i = 0; i < 4; ++i) {
+        if (ranges_overlap(outs[i], out_bytes[i], x, act) || ranges_overlap(outs[i], out_bytes[i], residual, act))
+            return PKV_ERR_INVALID_ARG;
+        for (int j = 0; j < i; ++j)
+            if (ranges_overlap(outs[i], out_bytes[i], outs[j], out_bytes[j])) return PKV_ERR_INVALID_ARG;
+    }
+    if (num_tokens == 0) return PKV_OK;
+    QkvPlan pl;
+    if (!qkv_plan(num_tokens, hidden, (int)N, &pl)) return PKV_ERR_CUDA;
+    pkv::QkvParams prm;
+    prm.x = static_cast<const __half*>(x);
+    prm.residual = static_cast<const __half*>(residual);
+    prm.gamma = static_cast<const __half*>(gamma);
+    prm.bias = static_cast<const __half*>(bias);
+    prm.residual_out = static_cast<__half*>(residual_out);
+    prm.q = static_cast<__half*>(q);
+    prm.k = static_cast<__half*>(k_new);
+    prm.v = static_cast<__half*>(v_new);
+    prm.T = num_tokens;
+    prm.H = hidden;
+    prm.N = (int32_t)N;
+    prm.q_cols = num_q_heads * head_dim;
+    prm.kv_cols = num_kv_heads * head_dim;
+    prm.kblocks = hidden / 64;
+    prm.split = pl.split;
+    prm.slab_blocks = pl.slab_blocks;
+    prm.eps = eps;
+    prm.prefetch_w = (flags & PKV_STEP_OVERLAP_PREVIOUS) ? 1 : 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return pl.mt == 1 ? launch_qkv<1>(pl, prm, w_qkv, st) : launch_qkv<2>(pl, prm, w_qkv, st);
 }
 
 }  // extern "C"

@@ -157,6 +157,53 @@ def test_fp8_scales_rejects_bad_arguments_on_host(kw, status):
     assert rc == status
 
 
+_QKV_BASE = 1 << 40                         # fake, 16-byte aligned, far apart
+_QKV_PTRS = {n: _QKV_BASE + (i << 32) for i, n in enumerate(
+    ("x", "residual", "gamma", "w", "bias", "res", "q", "k", "v"))}
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(w=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(v=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(q=_QKV_PTRS["q"] + 8), pkv.PKV_ERR_INVALID_ARG),        # 16-byte loads and stores
+    (dict(bias=_QKV_PTRS["bias"] + 4), pkv.PKV_ERR_INVALID_ARG),
+    (dict(res=_QKV_PTRS["residual"]), pkv.PKV_ERR_INVALID_ARG),   # in place: other CTAs still read it
+    (dict(q=_QKV_PTRS["x"] + 1024), pkv.PKV_ERR_INVALID_ARG),     # an output inside an input
+    (dict(k=_QKV_PTRS["q"] + 4096), pkv.PKV_ERR_INVALID_ARG),     # two outputs overlap
+    (dict(T=-1), pkv.PKV_ERR_INVALID_ARG),
+    (dict(Hkv=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(eps=-1e-6), pkv.PKV_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), pkv.PKV_ERR_INVALID_ARG),
+    (dict(flags=2), pkv.PKV_ERR_INVALID_ARG),
+    (dict(H=1000), pkv.PKV_ERR_UNSUPPORTED),                     # H a multiple of 64
+    (dict(H=10304), pkv.PKV_ERR_UNSUPPORTED),                    # above 8 slices of 20 blocks
+    (dict(D=12), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(T=65535 * 64 + 1), pkv.PKV_ERR_UNSUPPORTED),
+])
+def test_qkv_rejects_bad_arguments_on_host(kw, status):
+    a = dict(_QKV_PTRS, T=64, H=1536, Hq=12, Hkv=2, D=128, eps=1e-6, flags=0)
+    a.update(kw)
+    rc = pkv.load_library().fused_add_rmsnorm_qkv(
+        a["x"], a["residual"], a["gamma"], a["w"], a["bias"], a["res"], a["q"], a["k"], a["v"],
+        a["T"], a["H"], a["Hq"], a["Hkv"], a["D"], a["eps"], a["flags"], None)
+    assert rc == status
+
+
+def test_qkv_empty_batch_returns_before_any_cuda_call():
+    a = _QKV_PTRS
+    lib = pkv.load_library()
+    rc = lib.fused_add_rmsnorm_qkv(a["x"], a["residual"], a["gamma"], a["w"], None, a["res"],
+                                   a["q"], a["k"], a["v"], 0, 1536, 12, 2, 128, 1e-6, 0, None)
+    assert rc == pkv.PKV_OK
+    # empty per-token tensors may have null data pointers
+    rc = lib.fused_add_rmsnorm_qkv(0, 0, a["gamma"], a["w"], None, 0, 0, 0, 0, 0, 1536, 12, 2, 128, 1e-6, 0, None)
+    assert rc == pkv.PKV_OK
+    rc = lib.fused_add_rmsnorm_qkv(a["x"], a["residual"], 0, a["w"], None, a["res"],
+                                   a["q"], a["k"], a["v"], 0, 1536, 12, 2, 128, 1e-6, 0, None)
+    assert rc == pkv.PKV_ERR_INVALID_ARG
+
+
 def test_pages_head_counts_give_the_6x_kv_read_cut():
     """The GQA read saving the page quotes is Hq/Hkv under the byte model bench.py reports."""
     import json
