@@ -71,12 +71,22 @@ def step_bytes(w, lens, n_new):
     return a, cache_write_bytes(n_new, w.Hkv, w.head_dim, e)
 
 
+DECODE_SOURCES = ("cache_write.cuh", "decode_attention.cuh", "decode_balanced.cuh", "decode_page.cuh",
+                  "pkv_device.cuh")
+
+
 def kernel_source_digest() -> str:
+    """Hash of what the decode kernels are built from: their device headers and the launch-shape
+    constants in pagedkv.cu (worker warps, ring slots). Other kernels of the library do not enter."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_decode_gqa_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in DECODE_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    with open(os.path.join(csrc, "pagedkv.cu"), "rb") as f:
+        for line in f:
+            if b"PKV_BAL_" in line or b"constexpr int kStages" in line or b"constexpr int kConsumers" in line:
+                h.update(line)
     return h.hexdigest()[:16]
 
 
@@ -240,6 +250,9 @@ def qkv_bytes(T: int, H: int, N: int, bias: bool) -> int:
 def time_qkv_projection(w, device, stream, peak, seed=0):
     """fused_add_rmsnorm_qkv at the workload's model shape (H = Hq * D) for its batch, from a CUDA
     graph that rotates over enough weight replicas that W is read from HBM every launch."""
+    import torch
+
+    import paged_kv_decode_gqa_b200 as pkv
     Hq, Hkv, D, T = w.Hq, w.Hkv, w.head_dim, w.B
     H, N = Hq * D, (Hq + 2 * Hkv) * D
     d = W.make_qkv_inputs(T, H, Hq, Hkv, D, seed)

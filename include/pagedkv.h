@@ -266,7 +266,7 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
  * fp32 after the sum. The error is within 2^-10 * sum_k |w[n][k] y[t][k]|
  * plus the output rounding.
  *
- * Supported: H a multiple of 64 and at most 10240, D a multiple of 8,
+ * Supported: H a multiple of 64 and at most 8192, D a multiple of 8,
  * N <= 2^24, T <= 4194240; others return PKV_ERR_UNSUPPORTED. eps must be
  * finite and >= 0. T == 0 is a no-op (the per-token pointers may then be
  * NULL; gamma and w_qkv may not).

@@ -501,7 +501,7 @@ pkv_status check_device_scales(const float* k_scales, const float* v_scales, int
 // memory holds the activation slice.
 constexpr int kQkvStages1 = 4;
 constexpr int kQkvStages2 = 3;
-constexpr int kQkvMaxSplit = 8;                 // portable cluster size
+constexpr int kQkvMaxSplit = pkv::kQkvMaxCluster;   // portable cluster size
 template <int kMT>
 using QkvShapeT = pkv::QkvShape<kMT, kMT == 1 ? kQkvStages1 : kQkvStages2>;
 template <int kMT>
@@ -522,15 +522,15 @@ bool make_w_map(CUtensorMap* map, const void* w, int H, int N, int rows) {
 }
 
 struct QkvPlan {
-    int mt = 0, split = 0, slab_blocks = 0, ftiles = 0, ttiles = 0;
+    int mt = 0, split = 0, slab_blocks = 0, ftiles = 0, tiles_per_cta = 0, runs = 0, ttiles = 0;
     size_t smem = 0;
-    int64_t cost = 0;
+    double cost = 0;
 };
 
 template <int kMT>
 cudaLaunchConfig_t qkv_config(const QkvPlan& pl, cudaStream_t st, cudaLaunchAttribute (&attr)[2]) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(pl.ftiles * pl.split), (unsigned)pl.ttiles);
+    cfg.gridDim = dim3((unsigned)(pl.runs * pl.split), (unsigned)pl.ttiles);
     cfg.blockDim = dim3(QkvShapeT<kMT>::kThreads);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
@@ -545,10 +545,16 @@ cudaLaunchConfig_t qkv_config(const QkvPlan& pl, cudaStream_t st, cudaLaunchAttr
     return cfg;
 }
 
-// The plan for one tile height: as many slices of H per tile as fill the
-// SMs in one wave, at least as many as the activation slice needs, and one
-// that the device can schedule as a cluster. Its cost is the W bytes a CTA
-// streams times the waves. False if no split fits.
+// The best plan for one tile height. For each split of H (from the fewest
+// slices whose activations fit in shared memory up to the cluster limit) that
+// the device can schedule as a cluster, and each run length (feature tiles per
+// CTA), a cost in W-byte equivalents per CTA times the waves:
+//   run * tile rows * slice * 2      W streamed
+// + 7 * 64 * slice                   building the activation slice (measured:
+//                                    about 0.3 SM cycles an element, where W
+//                                    streams at about 25 bytes an SM cycle)
+// + run * 40000                      a tile's cluster reduction
+// Returns false if no split fits.
 template <int kMT>
 bool qkv_candidate(int T, int H, int N, int sms, QkvPlan* out) {
     using S = QkvShapeT<kMT>;
@@ -556,19 +562,21 @@ bool qkv_candidate(int T, int H, int N, int sms, QkvPlan* out) {
     auto kernel = qkv_kernel<kMT>();
     if (ensure_smem(kernel, (int)S::smem_bytes(S::kMaxSlabBlocks), &done) != cudaSuccess) return false;
     const int kb = H / 64;
-    QkvPlan pl;
-    pl.mt = kMT;
-    pl.ftiles = (N + S::kFT - 1) / S::kFT;
-    pl.ttiles = (T + S::kTT - 1) / S::kTT;
-    const int tiles = pl.ftiles * pl.ttiles;
+    const int ftiles = (N + S::kFT - 1) / S::kFT;
+    const int ttiles = (T + S::kTT - 1) / S::kTT;
     const int split_min = (kb + S::kMaxSlabBlocks - 1) / S::kMaxSlabBlocks;
     const int split_max = std::min(kQkvMaxSplit, kb);
-    if (split_min > split_max) return false;
-    for (int split = std::max(split_min, std::min(split_max, sms / std::max(tiles, 1))); split >= split_min;
-         --split) {
+    bool found = false;
+    for (int split = split_min; split <= split_max; ++split) {
+        QkvPlan pl;
+        pl.mt = kMT;
         pl.split = split;
         pl.slab_blocks = (kb + split - 1) / split;
         pl.smem = S::smem_bytes(pl.slab_blocks);
+        pl.ftiles = ftiles;
+        pl.ttiles = ttiles;
+        pl.tiles_per_cta = 1;
+        pl.runs = ftiles;
         cudaLaunchAttribute attr[2];
         cudaLaunchConfig_t cfg = qkv_config<kMT>(pl, nullptr, attr);
         int clusters = 0;
@@ -577,13 +585,24 @@ bool qkv_candidate(int T, int H, int N, int sms, QkvPlan* out) {
             continue;
         }
         if (clusters < 1) continue;
-        const int64_t ctas = (int64_t)tiles * split;
         const int64_t slots = std::max<int64_t>(1, std::min<int64_t>((int64_t)clusters * split, sms));
-        pl.cost = (ctas + slots - 1) / slots * S::kFT * pl.slab_blocks;
-        *out = pl;
-        return true;
+        for (int runs = ftiles; runs >= 1; --runs) {
+            const int per = (ftiles + runs - 1) / runs;
+            if ((ftiles + per - 1) / per != runs) continue;       // only the tightest run length per count
+            const int64_t ctas = (int64_t)runs * ttiles * split;
+            const int64_t waves = (ctas + slots - 1) / slots;
+            const double slice = 64.0 * pl.slab_blocks;
+            const double cost = (double)waves * (per * (double)S::kFT * slice * 2 + 7.0 * 64 * slice + per * 40000.0);
+            if (!found || cost < out->cost) {
+                pl.tiles_per_cta = per;
+                pl.runs = runs;
+                pl.cost = cost;
+                *out = pl;
+                found = true;
+            }
+        }
     }
-    return false;
+    return found;
 }
 
 bool qkv_plan(int T, int H, int N, QkvPlan* out) {
@@ -867,6 +886,8 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
     prm.kblocks = hidden / 64;
     prm.split = pl.split;
     prm.slab_blocks = pl.slab_blocks;
+    prm.ftiles = pl.ftiles;
+    prm.tiles_per_cta = pl.tiles_per_cta;
     prm.eps = eps;
     prm.prefetch_w = (flags & PKV_STEP_OVERLAP_PREVIOUS) ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

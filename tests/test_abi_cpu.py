@@ -177,7 +177,7 @@ _QKV_PTRS = {n: _QKV_BASE + (i << 32) for i, n in enumerate(
     (dict(eps=float("nan")), pkv.PKV_ERR_INVALID_ARG),
     (dict(flags=2), pkv.PKV_ERR_INVALID_ARG),
     (dict(H=1000), pkv.PKV_ERR_UNSUPPORTED),                     # H a multiple of 64
-    (dict(H=10304), pkv.PKV_ERR_UNSUPPORTED),                    # above 8 slices of 20 blocks
+    (dict(H=8256), pkv.PKV_ERR_UNSUPPORTED),                     # above 8 slices of 16 blocks
     (dict(D=12), pkv.PKV_ERR_UNSUPPORTED),
     (dict(T=65535 * 64 + 1), pkv.PKV_ERR_UNSUPPORTED),
 ])

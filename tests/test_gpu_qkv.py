@@ -81,8 +81,8 @@ def check(d, Hq, Hkv, D, eps=W.RMS_EPS, rows=None, flags=0, what=""):
     (64, 1536, 12, 2, 128),     # Qwen2.5-1.5B shape, one token tile
     (70, 1536, 12, 2, 128),     # a ragged second token tile
     (130, 512, 6, 1, 64),       # three token tiles, N = 512
-    (33, 3584, 28, 4, 128),     # Qwen2.5-7B shape, 256-row tiles
-    (3, 10240, 2, 1, 128),      # the largest H: eight slices of 20 blocks
+    (33, 3584, 28, 4, 128),     # Qwen2.5-7B shape: runs of several feature tiles per CTA
+    (3, 8192, 2, 1, 128),       # the largest H: eight slices of 16 blocks
     (9, 640, 1, 1, 8),          # N = 24: one partial weight tile
 ])
 @pytest.mark.parametrize("bias", [True, False])
