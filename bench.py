@@ -290,7 +290,7 @@ def time_qkv_projection(w, device, stream, peak, seed=0):
     return {"what": "fused_add_rmsnorm_qkv (residual add + RMSNorm + QKV projection, q/k/v out)",
             "T": T, "H": H, "N": N, "bias": True, "algorithmic_bytes": nbytes, "us": us,
             "achieved": nbytes / us / 1e3, "peak": peak, "unit": "GB/s", "frac": nbytes / us / 1e3 / peak,
-            "bound": "hbm", "launches": reps * R,
+            "bound": "hbm", "launches": reps * R, "plan": pkv.fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D),
             "l2": f"{R} weight replicas rotated ({R * N * H * 2 / 2**20:.0f} MiB), graph of {R} launches, "
                   "PKV_STEP_OVERLAP_PREVIOUS"}
 

@@ -283,6 +283,16 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
                                  int32_t num_kv_heads, int32_t head_dim, float eps,
                                  uint32_t flags, void* stream);
 
+/*
+ * fused_add_rmsnorm_qkv_plan -- the launch plan fused_add_rmsnorm_qkv uses on
+ * the current device for these sizes, for reports and tuning. Writes five
+ * int32 to plan (host memory): weight-tile rows, slices of the hidden size per
+ * cluster, feature tiles per CTA, CTAs, token tiles of 64. Host-only (queries
+ * the device's cluster occupancy); PKV_ERR_UNSUPPORTED as the projection.
+ */
+pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t* plan);
+
 /* Static text for a status code. Never NULL. */
 const char* pkv_status_string(pkv_status status);
 

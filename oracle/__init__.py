@@ -77,6 +77,9 @@ def _load():
         lib.oracle_f16_from_f64.restype = ctypes.c_uint16
         lib.oracle_add_rmsnorm_qkv.argtypes = [P, P, P, P, P, i32, i32, i32, ctypes.c_double, P, P]
         lib.oracle_add_rmsnorm_qkv.restype = i32
+        lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                             f32, i32, f32, f32]
+        lib.oracle_paged_prefill.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -275,3 +278,39 @@ def add_rmsnorm_qkv(x, residual, gamma, w_qkv, bias, eps, Hq, Hkv, D):
     k = qkv[:, Hq * D:(Hq + Hkv) * D].reshape(T, Hkv, D)
     v = qkv[:, (Hq + Hkv) * D:].reshape(T, Hkv, D)
     return res_out, q, k, v
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, softmax_scale, *,
+                  kv_dtype: str = "f16", k_scale: float = 1.0, v_scale: float = 1.0, return_lse: bool = False):
+    """Chunked prefill attention in float64 through the block tables (reading R12).
+
+    q: [total, Hq, D] float16, the n_b = query_start[b+1] - query_start[b] new tokens of each
+    sequence b, which are the last n_b of its context_lens[b] tokens (already in the cache).
+    k_cache, v_cache: [NB, bs, Hkv, D] float16 or uint8 (FP8). block_tables: [B, max_blocks]
+    int32. context_lens: [B] int32. query_start: [B + 1] int32. Returns out [total, Hq, D]
+    float64 (and lse [total, Hq]).
+    """
+    q = _c(q, np.float16)
+    fp8 = kv_dtype == "fp8"
+    cdt = np.uint8 if fp8 else np.float16
+    k_cache = _c(k_cache, cdt)
+    v_cache = _c(v_cache, cdt)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    qs = _c(query_start, np.int32)
+    total, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    B = cl.shape[0]
+    if D2 != D or v_cache.shape != k_cache.shape or qs.shape != (B + 1,) or qs[-1] != total:
+        raise ValueError("shape mismatch")
+    out = np.zeros((total, Hq, D), dtype=np.float64)
+    lse = np.zeros((total, Hq), dtype=np.float64)
+    rc = _load().oracle_paged_prefill(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(bt),
+                                      _ptr(cl), _ptr(qs), B, Hq, Hkv, D, bs, bt.shape[1], NB,
+                                      ctypes.c_float(softmax_scale), int(fp8), ctypes.c_float(k_scale),
+                                      ctypes.c_float(v_scale))
+    if rc == -1:
+        raise ValueError("block table entry outside the pool")
+    if rc != 0:
+        raise ValueError("bad lengths or head counts")
+    return (out, lse) if return_lse else out

@@ -50,6 +50,16 @@
  *       [0, Hq D) are the query heads, the next Hkv D the key heads, the
  *       last Hkv D the value heads, each head's D rows consecutive; no
  *       rotary embedding is applied (the pages name none).
+ *  Paged (chunked) prefill: the pages name prefill only as work the engine
+ *  does besides decode ("rvLLM 소개", §H100 SXM 80GB 직접 엔진 벤치마크:
+ *  the wall times include it), so:
+ *   R12 sequence b brings n_b = query_start[b+1] - query_start[b] query
+ *       tokens, the last n_b of its context_lens[b] = L_b tokens, whose K/V
+ *       are already in the cache; query i of b sits at position
+ *       p = L_b - n_b + i and attends causally to tokens [0, p] of b through
+ *       its block table, with R1's head map. q and out are [sum n_b, Hq, D]
+ *       with query_start [B+1] the prefix sums of n_b. n_b = 1 is decode;
+ *       n_b = L_b is a prefill from an empty cache.
  *
  * Build: gcc -O2 -fopenmp -fPIC -shared -ffp-contract=off (no fast-math).
  */
@@ -354,6 +364,56 @@ int oracle_paged_gqa_decode(double* out, double* lse, const uint16_t* q,
     free(ks);
     free(vs);
     return rc;
+}
+
+/* ------------------------------------------------------ paged prefill */
+
+/* Chunked prefill attention through the block tables (R12, R1-R5). out[i]
+ * (and lse[i], optional, [total, Hq]) for every query row i; per-tensor FP8
+ * scales as in decode. Returns 0, -1 for a table entry outside the pool, -2
+ * for bad lengths (n_b < 0, n_b > L_b, L_b beyond the table) or head counts. */
+int oracle_paged_prefill(double* out, double* lse, const uint16_t* q, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables,
+                         const int32_t* context_lens, const int32_t* query_start, int B, int Hq,
+                         int Hkv, int D, int block_size, int max_blocks_per_seq, int num_blocks,
+                         float softmax_scale, int kv_fp8, float k_scale, float v_scale) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || B < 0 || query_start[0] != 0) return -2;
+    for (int b = 0; b < B; ++b) {
+        int n = query_start[b + 1] - query_start[b], L = context_lens[b];
+        if (n < 0 || L < n || L > max_blocks_per_seq * block_size) return -2;
+    }
+    float* ks = (float*)malloc(sizeof(float) * (size_t)Hkv);
+    float* vs = (float*)malloc(sizeof(float) * (size_t)Hkv);
+    for (int g = 0; g < Hkv; ++g) { ks[g] = k_scale; vs[g] = v_scale; }
+    int status = 0;
+#pragma omp parallel for schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        int n = query_start[b + 1] - query_start[b], L = context_lens[b];
+        const int32_t* bt_row = block_tables + (int64_t)b * max_blocks_per_seq;
+        double* s = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        for (int i = 0; i < n; ++i) {
+            int64_t row = query_start[b] + i;
+            int pos = L - n + i;                    /* R12: this query's position */
+            const uint16_t* q_row = q + row * Hq * D;
+            for (int h = 0; h < Hq; ++h) {
+                double m, l;
+                double* o = out + (row * Hq + h) * D;
+                /* query row `row` is passed as sequence 0 of a one-row q */
+                if (attend_range(&m, &l, o, s, q_row, k_cache, v_cache, bt_row, 0, h, Hq, Hkv, D,
+                                 block_size, num_blocks, (double)softmax_scale, kv_fp8, ks, vs,
+                                 0, pos + 1)) {
+#pragma omp atomic write
+                    status = -1;
+                    continue;
+                }
+                if (lse) lse[row * Hq + h] = m + log(l);
+            }
+        }
+        free(s);
+    }
+    free(ks);
+    free(vs);
+    return status;
 }
 
 /* ------------------------------------------------ fused Add+RMSNorm+QKV */

@@ -50,6 +50,7 @@ _SIGNATURES = {
          _P, _sz, ctypes.c_uint32, _P], ctypes.c_int),
     "fused_add_rmsnorm_qkv": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _f32,
                                ctypes.c_uint32, _P], ctypes.c_int),
+    "fused_add_rmsnorm_qkv_plan": ([_i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -363,3 +364,10 @@ def fused_add_rmsnorm_qkv(x, residual, gamma, w_qkv, bias, residual_out, q, k_ne
         _ptr(x), _ptr(residual), _ptr(gamma), _ptr(w_qkv), _ptr(bias), _ptr(residual_out), _ptr(q),
         _ptr(k_new), _ptr(v_new), T, H, Hq, Hkv, D, float(eps), int(flags), _stream(stream)),
         "fused_add_rmsnorm_qkv")
+
+
+def fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D) -> dict:
+    """The launch plan of fused_add_rmsnorm_qkv for these sizes on the current device."""
+    plan = (ctypes.c_int32 * 5)()
+    _check(load_library().fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D, plan), "fused_add_rmsnorm_qkv_plan")
+    return dict(zip(("tile_rows", "slices", "tiles_per_cta", "ctas", "token_tiles"), list(plan)))

@@ -836,6 +836,24 @@ pkv_status paged_gqa_decode_step_fp8_scaled(
                      workspace, workspace_bytes, flags, stream);
 }
 
+pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t* plan) {
+    if (!plan || num_tokens <= 0 || hidden <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return PKV_ERR_INVALID_ARG;
+    const int64_t N = ((int64_t)num_q_heads + 2 * (int64_t)num_kv_heads) * head_dim;
+    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxSplit * 64 * QkvShapeT<1>::kMaxSlabBlocks ||
+        N > (1 << 24) || num_tokens > 65535 * 64)
+        return PKV_ERR_UNSUPPORTED;
+    QkvPlan pl;
+    if (!qkv_plan(num_tokens, hidden, (int)N, &pl)) return PKV_ERR_CUDA;
+    plan[0] = 128 * pl.mt;
+    plan[1] = pl.split;
+    plan[2] = pl.tiles_per_cta;
+    plan[3] = pl.runs * pl.split * pl.ttiles;
+    plan[4] = pl.ttiles;
+    return PKV_OK;
+}
+
 pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void* gamma, const void* w_qkv,
                                  const void* bias, void* residual_out, void* q, void* k_new, void* v_new,
                                  int32_t num_tokens, int32_t hidden, int32_t num_q_heads, int32_t num_kv_heads,

@@ -204,6 +204,19 @@ def test_qkv_empty_batch_returns_before_any_cuda_call():
     assert rc == pkv.PKV_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("args,status", [
+    ((64, 1536, 12, 2, 128, None), pkv.PKV_ERR_INVALID_ARG),
+    ((0, 1536, 12, 2, 128, "buf"), pkv.PKV_ERR_INVALID_ARG),
+    ((64, 1000, 12, 2, 128, "buf"), pkv.PKV_ERR_UNSUPPORTED),
+    ((64, 1536, 12, 2, 12, "buf"), pkv.PKV_ERR_UNSUPPORTED),
+])
+def test_qkv_plan_rejects_bad_arguments_on_host(args, status):
+    buf = (ctypes.c_int32 * 5)()
+    a = list(args)
+    a[5] = buf if a[5] == "buf" else None
+    assert pkv.load_library().fused_add_rmsnorm_qkv_plan(*a) == status
+
+
 def test_pages_head_counts_give_the_6x_kv_read_cut():
     """The GQA read saving the page quotes is Hq/Hkv under the byte model bench.py reports."""
     import json

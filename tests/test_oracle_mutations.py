@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_prefill as prefill_pins
 import test_oracle_qkv as qkv_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pkv_oracle.c")
@@ -52,6 +53,10 @@ MUTATIONS = {
     "weight_transposed": ("acc += oracle_f16_to_f64(wr[k]) * y[k];",
                           "acc += oracle_f16_to_f64(w[(int64_t)k * N + n]) * y[k];"),
     "bias_dropped": ("if (bias) acc += oracle_f16_to_f64(bias[n]);", ";"),
+    # paged prefill
+    "prefill_causal_off_by_one": ("0, pos + 1)) {", "0, pos + (pos == 0))) {"),
+    "prefill_position_from_start": ("int pos = L - n + i;", "int pos = i;"),
+    "prefill_rows_reversed": ("int64_t row = query_start[b] + i;", "int64_t row = query_start[b + 1] - 1 - i;"),
 }
 
 PIN_TESTS = [
@@ -71,6 +76,9 @@ PIN_TESTS = [
     lambda: qkv_pins.test_constant_row_and_eps(),
     lambda: qkv_pins.test_unit_rows_select_the_normalised_stream(),
     lambda: qkv_pins.test_qkv_split_follows_the_row_order(),
+    lambda: prefill_pins.test_one_query_per_sequence_is_decode(),
+    lambda: prefill_pins.test_matches_dense_causal_bruteforce([3, 1, 7, 40, 2]),
+    lambda: prefill_pins.test_later_positions_do_not_reach_earlier_queries(),
 ]
 
 
