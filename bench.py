@@ -295,6 +295,53 @@ def time_qkv_projection(w, device, stream, peak, seed=0):
                   "PKV_STEP_OVERLAP_PREVIOUS"}
 
 
+def prefill_flops(lens, n_new, Hq, D) -> int:
+    """Attention FLOPs of a chunked prefill: per query at position p, 2 D (p + 1) for the logits
+    and as many for the weighted values, per query head."""
+    total = 0
+    for L, n in zip(lens, n_new):
+        pos = np.arange(int(L) - int(n), int(L), dtype=np.int64)
+        total += int(4 * D * Hq * (pos + 1).sum())
+    return total
+
+
+def time_prefill(w, device, stream, peak_tflops, seed=0):
+    """paged_gqa_prefill_attention at the workload's head shape: 8 sequences append 512 tokens each
+    to contexts of 2048 (f16 cache), timed over back-to-back launches."""
+    import torch
+
+    import paged_kv_decode_gqa_b200 as pkv
+    B, n_new, L = 8, 512, 2048
+    pw = W.with_sizes(w, B=B, num_blocks=B * L // w.block_size + 64, ctx=("fixed", (L,) * B), kv_dtype="f16")
+    x = W.make_inputs(pw, seed, poison=False)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    qs = np.arange(0, (B + 1) * n_new, n_new, dtype=np.int32)
+    q = (np.random.default_rng(seed).standard_normal((B * n_new, w.Hq, w.head_dim), dtype=np.float32)
+         .astype(np.float16))
+    qd, kc, vc, bt, cl, qsd = t(q), t(x["k_pool"]), t(x["v_pool"]), t(x["block_tables"]), t(x["context_lens"]), t(qs)
+    out = torch.empty_like(qd)
+    call = lambda: pkv.paged_gqa_prefill_attention(out, qd, kc, vc, bt, cl, qsd, max_query_len=n_new,
+                                                   max_context_len=L, softmax_scale=float(x["softmax_scale"]),
+                                                   stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        reps = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1000 / reps
+    flops = prefill_flops([L] * B, [n_new] * B, w.Hq, w.head_dim)
+    tflops = flops / us / 1e6
+    return {"what": "paged_gqa_prefill_attention (chunked prefill, f16 cache)", "B": B, "new_tokens": n_new,
+            "context": L, "Hq": w.Hq, "Hkv": w.Hkv, "flops": flops, "us": us, "achieved": tflops,
+            "peak": peak_tflops, "unit": "TFLOP/s", "frac": tflops / peak_tflops, "bound": "tensor",
+            "launches": reps, "l2": "cache of 8 x 2048 tokens re-read by every chunk; L2-resident after the first"}
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -311,6 +358,8 @@ def parse_args(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="two launches per step (cache write, then attention) instead of the fused step")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip timing the chunked prefill attention at the workload's head shape")
     ap.add_argument("--no-qkv", action="store_true",
                     help="skip timing the fused add + RMSNorm + QKV projection at the workload's shape")
     ap.add_argument("--fp8-scales", default="tensor", choices=["tensor", "per-head"],
@@ -602,6 +651,9 @@ def run_ours(args):
             line["fp8_scales_kernel"] = scales_kernel
         if not args.no_qkv:
             line["qkv_kernel"] = time_qkv_projection(w, device, stream, peak, args.seed)
+        if not args.no_prefill:
+            line["prefill_kernel"] = time_prefill(w, device, stream, float(peaks.get("bf16_tflops", 1590.0)),
+                                                  args.seed)
         if e2e:
             line["e2e"] = e2e
         if world == 1 and args.cpu_baseline_s > 0:

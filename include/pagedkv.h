@@ -284,6 +284,42 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
                                  uint32_t flags, void* stream);
 
 /*
+ * paged_gqa_prefill_attention -- chunked prefill: many query tokens per
+ * sequence, each attending causally to the sequence's cached tokens through
+ * its block table.
+ *
+ * The pages name prefill as the engine's other attention work besides decode
+ * ("rvLLM 소개" (discuss.pytorch.kr), §H100 SXM 80GB 직접 엔진 벤치마크: the
+ * wall times include it), over the same paged cache (§PagedAttention과
+ * FlashAttention-3). This library's reading: sequence b brings
+ * n_b = query_start[b+1] - query_start[b] query tokens, the last n_b of its
+ * context_lens[b] = L_b tokens, whose K/V the cache write has already stored.
+ * Query i of b sits at position p = L_b - n_b + i and attends to positions
+ * [0, p]; query head h reads KV head h / (Hq / Hkv). With one query per
+ * sequence this is paged_gqa_decode_attention.
+ *
+ * Arguments (device pointers unless noted):
+ *   out, q          [total_queries, Hq, D] float16, rows in sequence order
+ *   k/v cache, block_tables, context_lens, block_size, num_blocks, FP8
+ *                   scales: as for paged_gqa_decode_attention (per-tensor scales)
+ *   query_start     [batch + 1] int32, query_start[0] = 0, non-decreasing,
+ *                   query_start[batch] = total_queries
+ *   max_query_len   host bound on n_b (sizes the grid); <= max_context_len
+ *   max_context_len host bound on L_b
+ * A sequence whose lengths are inconsistent on the device (n_b > L_b,
+ * L_b > max_context_len, n_b > max_query_len, rows outside [0,
+ * total_queries)) is flagged (PKV_DEVERR_CONTEXT_LEN) and its rows are left
+ * unwritten. No workspace; supported shapes as for decode.
+ */
+pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       const int32_t* query_start, int32_t batch, int32_t total_queries,
+                                       int32_t max_query_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                                       int32_t num_blocks, int32_t max_context_len, float softmax_scale,
+                                       int32_t kv_dtype, float k_scale, float v_scale, void* stream);
+
+/*
  * fused_add_rmsnorm_qkv_plan -- the launch plan fused_add_rmsnorm_qkv uses on
  * the current device for these sizes, for reports and tuning. Writes five
  * int32 to plan (host memory): weight-tile rows, slices of the hidden size per

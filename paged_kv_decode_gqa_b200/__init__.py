@@ -51,6 +51,8 @@ _SIGNATURES = {
     "fused_add_rmsnorm_qkv": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _f32,
                                ctypes.c_uint32, _P], ctypes.c_int),
     "fused_add_rmsnorm_qkv_plan": ([_i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "paged_gqa_prefill_attention": ([_P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                     _i32, _i32, _i32, _f32, _i32, _f32, _f32, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -371,3 +373,27 @@ def fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D) -> dict:
     plan = (ctypes.c_int32 * 5)()
     _check(load_library().fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D, plan), "fused_add_rmsnorm_qkv_plan")
     return dict(zip(("tile_rows", "slices", "tiles_per_cta", "ctas", "token_tiles"), list(plan)))
+
+
+def paged_gqa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start, *,
+                                max_query_len, max_context_len, softmax_scale, kv_dtype="f16",
+                                k_scale=1.0, v_scale=1.0, stream=None) -> None:
+    """Chunked prefill: query rows q [total, Hq, D] of each sequence (query_start [B+1] int32), the
+    last n_b tokens of its context, attending causally through the block tables; out [total, Hq, D]."""
+    _dense("out", out, "float16")
+    _dense("q", q, "float16")
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _dense(n, t, "float16", "uint8")
+    _dense("block_tables", block_tables, "int32")
+    _dense("context_lens", context_lens, "int32")
+    _dense("query_start", query_start, "int32")
+    total, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or query_start.shape[0] != B + 1:
+        raise ValueError("shape mismatch")
+    _check(load_library().paged_gqa_prefill_attention(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
+        B, total, int(max_query_len), Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
+        float(softmax_scale), kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _stream(stream)),
+        "paged_gqa_prefill_attention")

@@ -18,6 +18,7 @@
 #include "decode_balanced.cuh"
 #include "fp8_scales.cuh"
 #include "qkv_proj.cuh"
+#include "prefill_attention.cuh"
 
 namespace {
 
@@ -642,6 +643,22 @@ pkv_status launch_qkv(const QkvPlan& pl, const pkv::QkvParams& prm, const void* 
     return cudaLaunchKernelEx(&cfg, qkv_kernel<kMT>(), map, prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ paged prefill
+// 8 query tokens per CTA (one per consumer warp), an 8-page ring.
+constexpr int kPrefillConsumers = 8;
+constexpr int kPrefillStages = 8;
+
+template <bool kFp8>
+pkv_status launch_prefill(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
+                          int chunks, int Hkv, int B, cudaStream_t stream) {
+    using S = pkv::PrefillShape<kFp8, kPrefillConsumers, kPrefillStages>;
+    auto kernel = pkv::prefill_attention_kernel<kFp8, kPrefillConsumers, kPrefillStages>;
+    static unsigned long long done = 0;
+    if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
+    return launch_pdl(kernel, dim3((unsigned)chunks, Hkv, B), dim3(S::kThreads), S::kSmemBytes, stream, mk, mv,
+                      prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 bool ranges_overlap(const void* a, int64_t na, const void* b, int64_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return na > 0 && nb > 0 && x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
@@ -834,6 +851,51 @@ pkv_status paged_gqa_decode_step_fp8_scaled(
                      num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
                      softmax_scale, PKV_KV_FP8_E4M3, 1.f, 1.f, DeviceScales{k_scales, v_scales, scales_per_head},
                      workspace, workspace_bytes, flags, stream);
+}
+
+pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       const int32_t* query_start, int32_t batch, int32_t total_queries,
+                                       int32_t max_query_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                                       int32_t num_blocks, int32_t max_context_len, float softmax_scale,
+                                       int32_t kv_dtype, float k_scale, float v_scale, void* stream) {
+    if (total_queries < 0 || max_query_len < 0) return PKV_ERR_INVALID_ARG;
+    const bool any = batch > 0 && total_queries > 0 && max_query_len > 0;
+    {
+        const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens,
+                                                  any ? batch : 0, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                  max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                                                  kv_dtype, k_scale, v_scale, 0);
+        if (v != PKV_OK || !any) return v;
+    }
+    if (!query_start || (reinterpret_cast<uintptr_t>(query_start) & 3u)) return PKV_ERR_INVALID_ARG;
+    if (max_query_len > max_context_len) return PKV_ERR_INVALID_ARG;
+    const bool fp8 = kv_dtype == PKV_KV_FP8_E4M3;
+    pkv::PrefillParams prm{};
+    prm.out = static_cast<__half*>(out);
+    prm.q = static_cast<const __half*>(q);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.query_start = query_start;
+    prm.total = total_queries;
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.G = num_q_heads / num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.max_query_len = max_query_len;
+    prm.logit_scale_log2 = softmax_scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+    prm.out_scale = fp8 ? v_scale : 1.f;
+    CUtensorMap mk, mv;
+    if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
+        !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
+        return PKV_ERR_CUDA;
+    const int chunks = (max_query_len + kPrefillConsumers - 1) / kPrefillConsumers;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return fp8 ? launch_prefill<true>(prm, mk, mv, chunks, num_kv_heads, batch, st)
+               : launch_prefill<false>(prm, mk, mv, chunks, num_kv_heads, batch, st);
 }
 
 pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_t num_q_heads,

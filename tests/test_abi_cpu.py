@@ -217,6 +217,35 @@ def test_qkv_plan_rejects_bad_arguments_on_host(args, status):
     assert pkv.load_library().fused_add_rmsnorm_qkv_plan(*a) == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(qs=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(qs=A + 2), pkv.PKV_ERR_INVALID_ARG),
+    (dict(out=0), pkv.PKV_ERR_INVALID_ARG),
+    (dict(total=-1), pkv.PKV_ERR_INVALID_ARG),
+    (dict(maxq=5000), pkv.PKV_ERR_INVALID_ARG),           # above max_context_len
+    (dict(dtype=7), pkv.PKV_ERR_INVALID_ARG),
+    (dict(D=64), pkv.PKV_ERR_UNSUPPORTED),
+    (dict(Hq=36, Hkv=4), pkv.PKV_ERR_UNSUPPORTED),        # groups above 8
+    (dict(total=0), pkv.PKV_OK),                          # nothing to do
+])
+def test_prefill_rejects_bad_arguments_on_host(kw, status):
+    a = dict(out=A, q=A, k=A, v=A, bt=A, cl=A, qs=A, B=4, total=64, maxq=16, Hq=12, Hkv=2, D=128, bs=16,
+             mb=256, nb=1024, maxc=4096, scale=0.088, dtype=0)
+    a.update(kw)
+    rc = pkv.load_library().paged_gqa_prefill_attention(
+        a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["qs"], a["B"], a["total"], a["maxq"], a["Hq"],
+        a["Hkv"], a["D"], a["bs"], a["mb"], a["nb"], a["maxc"], a["scale"], a["dtype"], 1.0, 1.0, None)
+    assert rc == status
+
+
+def test_prefill_flops_closed_form():
+    """One sequence prefilled from an empty cache: sum over positions of 4 D Hq (p + 1)."""
+    import bench
+    L, Hq, D = 100, 12, 128
+    assert bench.prefill_flops([L], [L], Hq, D) == 4 * D * Hq * L * (L + 1) // 2
+    assert bench.prefill_flops([L], [1], Hq, D) == 4 * D * Hq * L            # decode
+
+
 def test_pages_head_counts_give_the_6x_kv_read_cut():
     """The GQA read saving the page quotes is Hq/Hkv under the byte model bench.py reports."""
     import json

@@ -1,0 +1,104 @@
+"""Parity of paged_gqa_prefill_attention (chunked prefill through the block tables) with the float64
+oracle, at the attention tolerance (2e-3 max-abs, 1e-2 of max |oracle|); FP8 on the same E4M3 bytes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_gqa_b200 as pkv
+import workloads as W
+from _gpu_helpers import assert_attention_close, dev, fp8_caches, host
+
+pytestmark = pytest.mark.gpu
+F16 = np.float16
+
+
+@pytest.fixture(autouse=True)
+def _clear_device_error():
+    pkv.pkv_device_error()
+    yield
+    torch.cuda.synchronize()
+
+
+def _case(name, seed, n_new, **sizes):
+    w = W.with_sizes(W.WORKLOADS[name], **sizes)
+    x = W.make_inputs(w, seed)                     # unused pool rows are NaN: never read
+    lens = x["context_lens"]
+    n = np.array([min(int(L), k) for L, k in zip(lens, n_new)], np.int32)
+    qs = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = np.random.default_rng(seed + 7).standard_normal((int(qs[-1]), w.Hq, w.head_dim)).astype(F16)
+    return w, x, q, qs
+
+
+def _run(w, x, q, qs, kv_dtype="f16", kc=None, vc=None):
+    out = torch.full(q.shape, float("nan"), dtype=torch.float16, device="cuda")
+    kc = x["k_pool"] if kc is None else kc
+    vc = x["v_pool"] if vc is None else vc
+    n = qs[1:] - qs[:-1]
+    pkv.paged_gqa_prefill_attention(out, dev(q), dev(kc), dev(vc), dev(x["block_tables"]), dev(x["context_lens"]),
+                                    dev(qs), max_query_len=max(int(n.max()), 1),
+                                    max_context_len=max(int(x["context_lens"].max()), 1),
+                                    softmax_scale=float(x["softmax_scale"]), kv_dtype=kv_dtype,
+                                    k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+    return host(out)
+
+
+def _oracle(w, x, q, qs, kv_dtype="f16", kc=None, vc=None):
+    return oracle.paged_prefill(q, x["k_pool"] if kc is None else kc, x["v_pool"] if vc is None else vc,
+                                x["block_tables"], x["context_lens"], qs, float(x["softmax_scale"]),
+                                kv_dtype=kv_dtype, k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+
+
+@pytest.mark.parametrize("name,n_new,sizes", [
+    ("qwen2.5-1.5b", [1] * 6, dict(B=6, num_blocks=1024)),                          # decode as prefill
+    ("qwen2.5-1.5b", [3, 1, 7, 40, 2, 17], dict(B=6, num_blocks=1024)),             # chunked, ragged chunks
+    ("qwen2.5-1.5b", [300] * 4, dict(B=4, num_blocks=1024, ctx=("uniform", 1, 300))),  # from an empty cache
+    ("qwen2.5-7b", [9, 0, 64, 33], dict(B=4, num_blocks=2048)),                      # G = 7, a sequence without queries
+    ("tiny", [17, 40], {}),
+])
+def test_prefill_parity_f16(name, n_new, sizes):
+    w, x, q, qs = _case(name, 3, n_new, **sizes)
+    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), f"{name} {n_new[:3]}")
+    assert pkv.pkv_device_error() == 0
+
+
+@pytest.mark.parametrize("n_new", [[1] * 5, [5, 30, 2, 64, 11]])
+def test_prefill_parity_fp8(n_new):
+    w, x, q, qs = _case("fp8-e4m3", 4, n_new, B=5, num_blocks=4096, ctx=("uniform", 70, 1500))
+    kq, vq = fp8_caches(x)
+    got = _run(w, x, q, qs, "fp8", kq, vq)
+    assert_attention_close(got, _oracle(w, x, q, qs, "fp8", kq, vq), f"fp8 {n_new}")
+    assert pkv.pkv_device_error() == 0
+
+
+def test_one_query_per_sequence_matches_decode():
+    w, x, q, qs = _case("qwen2.5-7b", 5, [1] * 6, B=6, num_blocks=2048)
+    got = _run(w, x, q, qs)
+    out = torch.empty(q.shape, dtype=torch.float16, device="cuda")
+    pkv.paged_gqa_decode_attention(out, dev(q), dev(x["k_pool"]), dev(x["v_pool"]), dev(x["block_tables"]),
+                                   dev(x["context_lens"]), max_context_len=int(x["context_lens"].max()),
+                                   softmax_scale=float(x["softmax_scale"]))
+    ref = _oracle(w, x, q, qs)
+    assert_attention_close(got, ref, "prefill n=1")
+    assert_attention_close(host(out), ref, "decode")
+
+
+def test_long_chunked_prefill():
+    """Two sequences append 256 tokens to contexts of up to 2048 (Qwen2.5-7B heads)."""
+    w, x, q, qs = _case("qwen2.5-7b", 6, [256, 256], B=2, num_blocks=1024, ctx=("uniform", 1024, 2048))
+    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "long chunked prefill")
+
+
+def test_inconsistent_lengths_are_flagged_not_faulted():
+    w, x, q, qs = _case("qwen2.5-1.5b", 8, [4, 4, 4], B=3, num_blocks=256, ctx=("fixed", (20, 3, 30)))
+    # sequence 1 has a 3-token context; ask for 4 queries by moving the boundaries
+    qs_bad = np.array([0, 4, 8, 12], np.int32)
+    q_bad = np.zeros((12, w.Hq, w.head_dim), F16)
+    out = torch.full(q_bad.shape, 7.0, dtype=torch.float16, device="cuda")
+    pkv.paged_gqa_prefill_attention(out, dev(q_bad), dev(x["k_pool"]), dev(x["v_pool"]), dev(x["block_tables"]),
+                                    dev(x["context_lens"]), dev(qs_bad), max_query_len=4, max_context_len=30,
+                                    softmax_scale=float(x["softmax_scale"]))
+    got = host(out)
+    assert pkv.pkv_device_error() & pkv.DEVERR_CONTEXT_LEN
+    assert (got[4:8] == 7.0).all()                  # the flagged sequence's rows are left alone
+    assert np.isfinite(got[:4]).all() and np.isfinite(got[8:]).all()
