@@ -1,7 +1,7 @@
 /*
  * pagedkv.h -- C ABI of the B200 (sm_100a) paged-KV decode library.
  *
- * Two operations of one decode step of a vLLM-style serving engine:
+ * The operations of one decode step of a vLLM-style serving engine:
  *
  *  1. paged_kv_cache_write ("reshape_and_cache"): scatter this step's new K/V
  *     vectors into their physical slots of the paged KV cache.
@@ -10,6 +10,12 @@
  *     through a PagedAttention block table, with an optional split-KV
  *     (flash-decoding) mode whose partial softmaxes are merged by the
  *     log-sum-exp rule inside the same launch.
+ *  3. paged_gqa_decode_step: 1 and 2 in one launch.
+ * and around them: fused_add_rmsnorm_qkv, the residual add, RMSNorm and QKV
+ * projection that produce the step's q and new K/V; paged_kv_fp8_scales and
+ * the *_fp8_scaled variants, FP8 caches with scales on the device; and
+ * paged_gqa_prefill_attention, many query tokens per sequence over the same
+ * paged cache (chunked prefill).
  *
  * Sources, cited by page title and section:
  *  - "rvLLM 소개" (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3:

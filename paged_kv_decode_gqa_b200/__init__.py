@@ -8,12 +8,14 @@ library's kernels. There is no CPU fallback; importing this package fails if
 the library has not been built (``python -m paged_kv_decode_gqa_b200.build``).
 
 Tensors are torch CUDA tensors used as plain device memory:
-  q, out            [B, Hq, D]              float16
+  q, out            [B, Hq, D]              float16 (prefill: [total queries, Hq, D])
   k_cache, v_cache  [NB, block_size, Hkv, D] float16, or uint8 (FP8 E4M3 codes)
   k_new, v_new      [T, Hkv, D]             float16
   block_tables      [B, max_blocks]         int32
   context_lens      [B]                     int32
   slot_mapping      [T]                     int64
+  query_start       [B + 1]                 int32 (prefill)
+  x, residual       [T, H]                  float16 (QKV projection; w_qkv [N, H], gamma [H])
 """
 from __future__ import annotations
 
