@@ -649,11 +649,19 @@ def run_ours(args):
         }
         if scales_kernel:
             line["fp8_scales_kernel"] = scales_kernel
+        # side measurements of the other kernels: a failure is reported in its key, and the
+        # step's line is still printed
+        side = []
         if not args.no_qkv:
-            line["qkv_kernel"] = time_qkv_projection(w, device, stream, peak, args.seed)
+            side.append(("qkv_kernel", lambda: time_qkv_projection(w, device, stream, peak, args.seed)))
         if not args.no_prefill:
-            line["prefill_kernel"] = time_prefill(w, device, stream, float(peaks.get("bf16_tflops", 1590.0)),
-                                                  args.seed)
+            side.append(("prefill_kernel", lambda: time_prefill(
+                w, device, stream, float(peaks.get("bf16_tflops", 1590.0)), args.seed)))
+        for key, measure in side:
+            try:
+                line[key] = measure()
+            except Exception as exc:  # noqa: BLE001 -- reported, never silent
+                line[key] = {"error": f"{type(exc).__name__}: {exc}"}
         if e2e:
             line["e2e"] = e2e
         if world == 1 and args.cpu_baseline_s > 0:
