@@ -152,3 +152,20 @@ def test_bad_lengths_are_rejected():
     with pytest.raises(ValueError):
         oracle.paged_prefill(q6, x["k_pool"], x["v_pool"], x["block_tables"], x["context_lens"], bad,
                              float(x["softmax_scale"]))
+
+
+def test_lse_matches_dense_logsumexp():
+    """The returned log-sum-exp is that of the masked logits (natural log, scaled logits)."""
+    w, x, q, qs = _case(10, [4, 9, 1, 30, 6])
+    _, lse = _prefill(w, x, q, qs, return_lse=True)
+    G = w.Hq // w.Hkv
+    for b in range(w.B):
+        L, n = int(x["context_lens"][b]), int(qs[b + 1] - qs[b])
+        t = np.arange(L)
+        K = x["k_pool"][x["block_tables"][b, t // w.block_size], t % w.block_size].astype(np.float64)
+        for i in range(n):
+            pos = L - n + i
+            for h in range(w.Hq):
+                s = float(x["softmax_scale"]) * (K[:pos + 1, h // G] @ q[qs[b] + i, h].astype(np.float64))
+                want = s.max() + np.log(np.exp(s - s.max()).sum())
+                assert abs(lse[qs[b] + i, h] - want) <= 1e-12 * max(1.0, abs(want))
