@@ -94,6 +94,14 @@ typedef enum {
 
 /* flags of paged_gqa_decode_step */
 #define PKV_STEP_OVERLAP_PREVIOUS 0x1u
+/* Failure-detection self-test of paged_gqa_decode_step (never needed in
+ * service): worker warp 0 of the persistent grid issues none of its page
+ * loads, so its first barrier wait can never complete, and every barrier
+ * wait of the launch gives up after 2 ms instead of one second. The launch
+ * ends normally with PKV_DEVERR_WAIT_TIMEOUT set; that worker's share of the
+ * output is left unwritten, no copy is left in flight, and the workspace
+ * must be zero-filled again before its next use (see below). */
+#define PKV_STEP_SELFTEST_WAIT_TIMEOUT 0x100u
 
 /* Bits of the device error word (pkv_device_error). */
 #define PKV_DEVERR_CONTEXT_LEN   0x1u  /* a context length exceeded max_context_len or the
@@ -175,9 +183,12 @@ int32_t paged_gqa_decode_suggest_partition(int32_t batch, int32_t num_kv_heads,
  *   M = max m_p, w_p = l_p * exp(m_p - M), out = sum w_p o_p / sum w_p.
  *   `workspace` must then hold paged_gqa_decode_workspace_size(...) bytes,
  *   256-byte aligned, and must be ZERO-FILLED before its first use; every
- *   call leaves it ready for the next one (its counters back at zero), so a
- *   workspace is allocated and cleared once and reused. Calls that share a
- *   workspace must not run concurrently on different streams.
+ *   call that completes without a device error leaves it ready for the next
+ *   one (its counters back at zero), so a workspace is allocated and cleared
+ *   once and reused. A call that ended with a barrier-wait timeout
+ *   (PKV_DEVERR_WAIT_TIMEOUT) can leave counters set: zero-fill the
+ *   workspace again before reusing it. Calls that share a workspace must not
+ *   run concurrently on different streams.
  *
  * max_context_len must be >= every context_lens[b] (larger lengths are
  * clamped and flagged) and <= max_blocks_per_seq * block_size.
@@ -214,7 +225,8 @@ pkv_status paged_gqa_decode_attention(void* out, const void* q,
  * first use). Batches whose tables do not fit the kernel's shared memory
  * (above 8192 sequences) return PKV_ERR_UNSUPPORTED.
  *
- * flags: 0, or PKV_STEP_OVERLAP_PREVIOUS. The kernel is launched with
+ * flags: 0, or PKV_STEP_OVERLAP_PREVIOUS (PKV_STEP_SELFTEST_WAIT_TIMEOUT may
+ * be added for the self-test above). The kernel is launched with
  * programmatic dependent launch, so it may start while the previous launch
  * in `stream` finishes. By default it waits for that launch before reading
  * any input. With PKV_STEP_OVERLAP_PREVIOUS it first reads context_lens,
@@ -347,9 +359,9 @@ pkv_status pkv_device_error(uint32_t* flags);
 
 /*
  * Size of the library-owned split-KV scratch used by
- * paged_gqa_decode_attention_static_workspace (8 MiB per GPU).
+ * paged_gqa_decode_attention_static_workspace (16 MiB per GPU).
  */
-#define PKV_STATIC_WORKSPACE_BYTES (8u << 20)
+#define PKV_STATIC_WORKSPACE_BYTES (16u << 20)
 
 /*
  * paged_gqa_decode_attention_static_workspace -- the same attention as
@@ -361,22 +373,28 @@ pkv_status pkv_device_error(uint32_t* flags);
  * recorded into a CUDA graph where cudaMalloc must not be called, or a
  * foreign-language caller with no access to the process's allocator.
  *
- * Arguments are those of paged_gqa_decode_attention without the workspace.
- * The split-KV scratch is a fixed PKV_STATIC_WORKSPACE_BYTES array inside the
- * library (a file-scope __device__ array: every GPU that loads the library
- * holds it until the process exits). Nothing is allocated and no allocating
- * library routine is called.
- *  - Sizes whose split-KV scratch, paged_gqa_decode_workspace_size(...),
- *    exceeds PKV_STATIC_WORKSPACE_BYTES are rejected with PKV_ERR_WORKSPACE
- *    before any launch; single-pass calls need no scratch.
+ * Arguments are those of paged_gqa_decode_attention without the workspace,
+ * and every plan is served: PKV_PARTITION_AUTO (the balanced kernel, or the
+ * fixed partitions it falls back to for very large batches), fixed
+ * partitions, and the single pass. The scratch is a fixed
+ * PKV_STATIC_WORKSPACE_BYTES array inside the library (a file-scope
+ * __device__ array: every GPU that loads the library holds it until the
+ * process exits). Nothing is allocated and no allocating library routine is
+ * called.
+ *  - A plan whose scratch exceeds PKV_STATIC_WORKSPACE_BYTES is rejected
+ *    with PKV_ERR_WORKSPACE before any launch. The balanced plan needs two
+ *    partial results per worker warp of the persistent grid (about 10 MiB on
+ *    a 148-SM B200 with an FP8 cache); fixed partitions need
+ *    paged_gqa_decode_workspace_size(...) bytes; a single pass needs none.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture on the device.
  *  - Every call on a device shares the one array, which keeps the previous
  *    call's contents; each call clears the part that must start at zero (its
- *    partition counters) on `stream` before launching. Calls whose execution
- *    overlaps on the GPU (other streams, other threads) race on the array and
- *    give undefined results: serialise them.
+ *    merge counters) on `stream` before launching, so a call that ended with
+ *    a device error (PKV_DEVERR_*) does not affect the next one. Calls whose
+ *    execution overlaps on the GPU (other streams, other threads) race on
+ *    the array and give undefined results: serialise them.
  */
 pkv_status paged_gqa_decode_attention_static_workspace(
     void* out, const void* q, const void* k_cache, const void* v_cache,

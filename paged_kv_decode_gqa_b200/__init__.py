@@ -89,6 +89,7 @@ PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_WORKSPACE, PKV_ERR_CUD
 PKV_KV_F16, PKV_KV_FP8_E4M3 = 0, 1
 PKV_PARTITION_AUTO = -1         # partition_tokens: the library's load-balanced plan
 PKV_STEP_OVERLAP_PREVIOUS = 0x1  # paged_gqa_decode_step flag (see include/pagedkv.h)
+PKV_STEP_SELFTEST_WAIT_TIMEOUT = 0x100  # self-test: one worker loads nothing, its wait runs out
 DEVERR_CONTEXT_LEN, DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_WAIT_TIMEOUT, DEVERR_SCALE = 0x1, 0x2, 0x4, 0x8, 0x10
 _KV_DTYPES = {"f16": PKV_KV_F16, "fp8": PKV_KV_FP8_E4M3}
 
@@ -222,7 +223,7 @@ def pkv_device_error() -> int:
 
 
 # Size of the library's own split-KV scratch (PKV_STATIC_WORKSPACE_BYTES).
-STATIC_WORKSPACE_BYTES = 8 << 20
+STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 def paged_gqa_decode_attention_static_workspace(out, q, k_cache, v_cache, block_tables,

@@ -54,6 +54,10 @@ struct BalancedParams {
     const float* k_scales;        // FP8 device scales [1] or [Hkv], or null: then for KV head g the
     const float* v_scales;        // logit scale is logit_scale_log2 * k_scales[g], the output scale
     int32_t scales_per_head;      // v_scales[g], and the new token is quantised with them
+    // failure-detection self-test: this worker (-1: none) issues none of its page loads, so its
+    // first barrier wait never completes; every wait of the launch gives up after wait_limit_ns
+    int32_t stall_worker;
+    uint64_t wait_limit_ns;
 };
 
 constexpr int kMergeFloats = 32 * 8 + 16;     // per warp: weights of 32 items x 8 heads, M, L
@@ -228,6 +232,8 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     load_window(0, win_phys, win_head);
     load_window(1, nxt_phys, nxt_head);
     const uint64_t policy = l2_evict_first_policy();
+    const bool stalled = worker == p.stall_worker;   // self-test: this worker loads nothing
+    int issued = 0;                                  // units [0, issued) have their loads in flight or landed
 
     // Issues the TMA loads of unit t (t < n) into slot t % kStages; whole warp.
     auto issue = [&](int t) {
@@ -240,6 +246,8 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         int pb = __shfl_sync(0xffffffffu, win_phys, t & 31);
         const int hg = __shfl_sync(0xffffffffu, win_head, t & 31);
+        if (stalled) return;
+        issued = t + 1;
         if (lane == 0) {
             if (pb < 0 || pb >= p.num_blocks) {     // outside the pool: reads as zeros
                 flag_error(PKV_DEVERR_BLOCK_ID);
@@ -481,13 +489,28 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         __syncwarp();
     };
 
+    // A wait that ran out (flagged by mbar_wait) ends this worker: first it
+    // waits, again with the limit, for the loads it issued after unit `lost`,
+    // so that no copy into its ring is in flight when it returns. Its piece
+    // is neither written nor merged; the caller learns of it from the
+    // device error word, and the workspace's tickets must be cleared.
+    auto drain_after = [&](int lost) {
+        for (int u = lost + 1; u < issued; ++u)
+            mbar_wait(full_bar(u % kStages), (u / kStages) & 1, p.wait_limit_ns);
+    };
     for (int t = 0; t < n; ++t) {
         const int s = t % kStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (t / kStages) & 1))) return;
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (t / kStages) & 1, p.wait_limit_ns))) {
+            drain_after(t);
+            return;
+        }
         if (kPagePairs && j + 1 < nb && t + 1 < n) {
             // pages t and t + 1 are consecutive pages of one segment: one softmax step
             const int s2 = (t + 1) % kStages;
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s2), ((t + 1) / kStages) & 1))) return;
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s2), ((t + 1) / kStages) & 1, p.wait_limit_ns))) {
+                drain_after(t + 1);
+                return;
+            }
             const int valid_b = j + 1 == nb - 1 ? lens[b] - (j + 1) * kPageRows : kPageRows;
             if constexpr (kFuseWrite) {
                 if (j + 1 == nb - 1) write_new_token(s2, j + 1);   // page B holds position L - 1

@@ -54,6 +54,8 @@ constexpr int kBalStagesF16 = PKV_BAL_STAGES_F16;
 constexpr int kBalStagesFp8 = PKV_BAL_STAGES_FP8;
 constexpr int kBalMaxBatch = 8192;        // unit-order tables must fit in shared memory
 constexpr int kBalMinUnits = 4;           // pages per worker at least (small batches)
+// Barrier-wait limit of a launch under PKV_STEP_SELFTEST_WAIT_TIMEOUT.
+constexpr uint64_t kSelftestWaitLimitNs = 2000000ull;   // 2 ms
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -244,7 +246,7 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
                            int32_t Hq, int32_t Hkv, int32_t max_blocks_per_seq, int32_t num_blocks,
                            int32_t max_context_len, float softmax_scale, float k_scale, float v_scale,
                            const DeviceScales& ds, void* workspace, size_t workspace_bytes,
-                           bool overlap_previous, cudaStream_t st) {
+                           bool overlap_previous, cudaStream_t st, bool selftest_stall = false) {
     const BalancedLayout bl = balanced_layout((int64_t)grid * bal_warps(fp8), batch, Hkv);
     if (!workspace || workspace_bytes < bl.total) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
@@ -279,6 +281,8 @@ pkv_status launch_balanced(bool fp8, int grid, const void* k_new, const void* v_
     bp.k_scales = fp8 ? ds.k : nullptr;
     bp.v_scales = fp8 ? ds.v : nullptr;
     bp.scales_per_head = ds.per_head;
+    bp.stall_worker = selftest_stall ? 0 : -1;
+    bp.wait_limit_ns = selftest_stall ? kSelftestWaitLimitNs : pkv::kWaitLimitNs;
     CUtensorMap mk, mv;
     if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, Hkv) ||
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, Hkv))
@@ -304,6 +308,51 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t npa
     w.count = w.l + align256(rows * sizeof(float));
     w.total = w.count + align256(B * Hkv * sizeof(unsigned int));
     return w;
+}
+
+// The plan paged_gqa_decode_attention runs for these sizes on the current
+// device, and the scratch it needs: the balanced kernel for
+// PKV_PARTITION_AUTO when the batch's tables fit (else fixed partitions of
+// the suggested size); fixed partitions, rounded up to whole pages, when
+// partition_tokens > 0, a single pass when one partition covers the longest
+// context. `zero_off`/`zero_bytes` is the part of the scratch that must be
+// zero when a call starts (the merge counters).
+struct AttnPlan {
+    bool balanced = false;
+    int grid = 0;
+    int32_t partition = 0;
+    int nparts = 1;
+    size_t ws_bytes = 0, zero_off = 0, zero_bytes = 0;
+};
+
+AttnPlan plan_attention(bool fp8, int32_t batch, int32_t Hq, int32_t Hkv, int32_t max_blocks_per_seq,
+                        int32_t max_context_len, int32_t partition_tokens) {
+    AttnPlan pl;
+    if (partition_tokens == PKV_PARTITION_AUTO) {
+        pl.grid = !use_balanced(batch, Hkv, max_blocks_per_seq) ? 0
+                  : fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
+        if (pl.grid > 0) {
+            const BalancedLayout bl = balanced_layout((int64_t)pl.grid * bal_warps(fp8), batch, Hkv);
+            pl.balanced = true;
+            pl.ws_bytes = bl.total;
+            pl.zero_off = bl.count;
+            pl.zero_bytes = bl.total - bl.count;
+            return pl;
+        }
+        partition_tokens = paged_gqa_decode_suggest_partition(batch, Hkv, max_context_len, kPageRows, 0);
+    }
+    int32_t P = partition_tokens;
+    if (P == 0 || P >= max_context_len) P = std::max(max_context_len, 1);
+    P = (P + kPageRows - 1) / kPageRows * kPageRows;
+    pl.partition = P;
+    pl.nparts = std::max(1, (max_context_len + P - 1) / P);
+    if (pl.nparts > 1) {
+        const WorkspaceLayout wl = workspace_layout(batch, Hq, Hkv, pl.nparts);
+        pl.ws_bytes = wl.total;
+        pl.zero_off = wl.count;
+        pl.zero_bytes = wl.total - wl.count;
+    }
+    return pl;
 }
 
 // Host-side argument checks shared by the attention entry points (PKV_OK for
@@ -406,24 +455,16 @@ pkv_status attention_impl(void* out, const void* q, const void* k_cache, const v
 
     const float log2e = 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (partition_tokens == PKV_PARTITION_AUTO) {
-        const int grid = !use_balanced(batch, num_kv_heads, max_blocks_per_seq) ? 0
-                         : fp8 ? balanced_grid<true>(batch) : balanced_grid<false>(batch);
-        if (grid > 0) {
-            return launch_balanced(fp8, grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
-                                   context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
-                                   num_blocks, max_context_len, softmax_scale, k_scale, v_scale, ds,
-                                   workspace, workspace_bytes, false, st);
-        }
-        partition_tokens = paged_gqa_decode_suggest_partition(batch, num_kv_heads, max_context_len,
-                                                              kPageRows, 0);
+    const AttnPlan plan = plan_attention(fp8, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
+                                         max_context_len, partition_tokens);
+    if (plan.balanced) {
+        return launch_balanced(fp8, plan.grid, nullptr, nullptr, out, q, k_cache, v_cache, block_tables,
+                               context_lens, batch, num_q_heads, num_kv_heads, max_blocks_per_seq,
+                               num_blocks, max_context_len, softmax_scale, k_scale, v_scale, ds,
+                               workspace, workspace_bytes, false, st);
     }
-
-    // plan: a partition covering the longest context is a single pass
-    int32_t P = partition_tokens;
-    if (P == 0 || P >= max_context_len) P = std::max(max_context_len, 1);
-    P = (P + kPageRows - 1) / kPageRows * kPageRows;
-    const int nparts = std::max(1, (max_context_len + P - 1) / P);
+    const int32_t P = plan.partition;
+    const int nparts = plan.nparts;
 
     pkv::DecodeParams prm{};
     prm.out = static_cast<__half*>(out);
@@ -470,7 +511,7 @@ pkv_status step_impl(void* out, const void* q, const void* k_new, const void* v_
                                  float softmax_scale, int32_t kv_dtype, float k_scale, float v_scale,
                                  const DeviceScales& ds, void* workspace, size_t workspace_bytes,
                                  uint32_t flags, void* stream) {
-    if (flags & ~PKV_STEP_OVERLAP_PREVIOUS) return PKV_ERR_INVALID_ARG;
+    if (flags & ~(PKV_STEP_OVERLAP_PREVIOUS | PKV_STEP_SELFTEST_WAIT_TIMEOUT)) return PKV_ERR_INVALID_ARG;
     const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                               num_q_heads, num_kv_heads, head_dim, block_size,
                                               max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
@@ -484,7 +525,8 @@ pkv_status step_impl(void* out, const void* q, const void* k_new, const void* v_
     return launch_balanced(fp8, grid, k_new, v_new, out, q, k_cache, v_cache, block_tables, context_lens,
                            batch, num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks,
                            max_context_len, softmax_scale, k_scale, v_scale, ds, workspace, workspace_bytes,
-                           (flags & PKV_STEP_OVERLAP_PREVIOUS) != 0, static_cast<cudaStream_t>(stream));
+                           (flags & PKV_STEP_OVERLAP_PREVIOUS) != 0, static_cast<cudaStream_t>(stream),
+                           (flags & PKV_STEP_SELFTEST_WAIT_TIMEOUT) != 0);
 }
 
 // Validates a device-scale pair (a per-head set needs num_kv_heads entries).
@@ -1007,30 +1049,30 @@ extern "C" pkv_status paged_gqa_decode_attention_static_workspace(
     int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
     int32_t num_blocks, int32_t max_context_len, float softmax_scale, int32_t kv_dtype,
     float k_scale, float v_scale, int32_t partition_tokens, void* stream) {
-    // Split-KV needs scratch only when more than one partition covers the
-    // longest context (the same rule paged_gqa_decode_attention applies).
-    const bool split = partition_tokens > 0 && partition_tokens < max_context_len;
+    const pkv_status v = check_attention_args(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                              num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+                                              kv_dtype, k_scale, v_scale, partition_tokens);
+    if (v != PKV_OK || batch == 0) return v;
+    // The scratch of the plan paged_gqa_decode_attention will run (the same
+    // rule it applies): the balanced kernel's piece slots and tickets for
+    // PKV_PARTITION_AUTO, the partitions' results and counters for fixed
+    // partitions, nothing for a single pass.
+    const AttnPlan plan = plan_attention(kv_dtype == PKV_KV_FP8_E4M3, batch, num_q_heads, num_kv_heads,
+                                         max_blocks_per_seq, max_context_len, partition_tokens);
     void* ws = nullptr;
     size_t ws_bytes = 0;
-    if (split && batch > 0 && num_kv_heads > 0 && num_q_heads > 0 && block_size > 0 &&
-        partition_tokens % block_size == 0) {
-        ws_bytes = paged_gqa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
-                                                   max_context_len, partition_tokens);
-        if (ws_bytes > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;
-        if (ws_bytes > 0) {
-            ws = static_workspace_address();
-            if (!ws) return PKV_ERR_CUDA;
-            // the previous call may have left other data where this call's
-            // partition counters go: clear them, in stream order
-            const int32_t P = (partition_tokens + kPageRows - 1) / kPageRows * kPageRows;
-            const int nparts = std::max(1, (max_context_len + P - 1) / P);
-            const WorkspaceLayout wl = workspace_layout(batch, num_q_heads, num_kv_heads, nparts);
-            if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + wl.count, 0,
-                                (size_t)batch * num_kv_heads * sizeof(unsigned int),
-                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
-                return PKV_ERR_CUDA;
-            ws_bytes = PKV_STATIC_WORKSPACE_BYTES;
-        }
+    if (plan.ws_bytes > 0) {
+        if (plan.ws_bytes > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;
+        ws = static_workspace_address();
+        if (!ws) return PKV_ERR_CUDA;
+        // the previous call may have left other data where this call's
+        // counters go: clear them, in stream order
+        if (plan.zero_bytes > 0 &&
+            cudaMemsetAsync(static_cast<uint8_t*>(ws) + plan.zero_off, 0, plan.zero_bytes,
+                            static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        ws_bytes = PKV_STATIC_WORKSPACE_BYTES;
     }
     return paged_gqa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                       num_q_heads, num_kv_heads, head_dim, block_size,

@@ -77,15 +77,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // one second
+
 // Waits until the phase of `bar` with parity `parity` has completed. Gives up
-// after about one second, flags PKV_DEVERR_WAIT_TIMEOUT and returns false, so
-// that a lost arrival ends the kernel with an error instead of a hang.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// after `limit_ns` (one second by default), flags PKV_DEVERR_WAIT_TIMEOUT and
+// returns false, so that a lost arrival ends the kernel with an error instead
+// of a hang.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > 1000000000ull) {
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) {
             flag_error(PKV_DEVERR_WAIT_TIMEOUT);
             return false;
         }

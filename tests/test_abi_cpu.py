@@ -255,3 +255,39 @@ def test_pages_head_counts_give_the_6x_kv_read_cut():
     grouped = bench.kv_bytes(lens, g["Hkv"], 128, 2)
     per_query_head = bench.kv_bytes(lens, g["Hq"], 128, 2)
     assert per_query_head / grouped == g["kv_bandwidth_reduction"]
+
+
+def test_header_macros_match_the_binding():
+    text = open(HEADER).read()
+    macros = {m: int(v, 0) for m, v in re.findall(r"#define\s+(PKV_\w+)\s+\(?([0-9x]+)u?\)?", text)}
+    m = re.search(r"#define\s+PKV_STATIC_WORKSPACE_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert pkv.STATIC_WORKSPACE_BYTES == int(m.group(1)) << int(m.group(2))
+    assert macros["PKV_STEP_OVERLAP_PREVIOUS"] == pkv.PKV_STEP_OVERLAP_PREVIOUS
+    assert macros["PKV_STEP_SELFTEST_WAIT_TIMEOUT"] == pkv.PKV_STEP_SELFTEST_WAIT_TIMEOUT
+    assert macros["PKV_DEVERR_WAIT_TIMEOUT"] == pkv.DEVERR_WAIT_TIMEOUT
+
+
+def _step(flags, **kw):
+    a = dict(out=A, q=A, kn=A, vn=A, k=A, v=A, bt=A, cl=A, B=2, Hq=12, Hkv=2, D=128, bs=16, mb=4, NB=64,
+             maxlen=40, scale=0.088, dt=0, ks=1.0, vs=1.0, ws=0, wsb=0)
+    a.update(kw)
+    return pkv.load_library().paged_gqa_decode_step(
+        a["out"], a["q"], a["kn"], a["vn"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["Hq"], a["Hkv"],
+        a["D"], a["bs"], a["mb"], a["NB"], a["maxlen"], a["scale"], a["dt"], a["ks"], a["vs"], a["ws"],
+        a["wsb"], flags, None)
+
+
+@pytest.mark.parametrize("flags", [0x2, 0x200, 0x80000000])
+def test_step_rejects_unknown_flags_on_host(flags):
+    assert _step(flags) == pkv.PKV_ERR_INVALID_ARG
+
+
+def test_static_workspace_entry_rejects_bad_arguments_on_host():
+    lib = pkv.load_library()
+    call = lambda **kw: lib.paged_gqa_decode_attention_static_workspace(
+        *[kw.get(k, A) for k in ("out", "q", "k", "v", "bt", "cl")], kw.get("B", 2), 12, 2, kw.get("D", 128), 16,
+        4, 64, 40, 0.088, 0, 1.0, 1.0, kw.get("P", 0), None)
+    assert call(q=0) == pkv.PKV_ERR_INVALID_ARG
+    assert call(D=64) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(P=20) == pkv.PKV_ERR_INVALID_ARG
+    assert call(B=0) == pkv.PKV_OK
