@@ -10,8 +10,16 @@ the Qwen2.5 serving workloads ("rvLLM 소개" (discuss.pytorch.kr),
 §PagedAttention과 FlashAttention-3 and §H100 SXM 80GB 직접 엔진 벤치마크),
 resident in HBM before timing. The K timed steps are replayed from CUDA
 graphs, as the serving engine replays its decode step (same page, §CUDA
-그래프 리플레이); consecutive steps read different replicas of the KV pool so
-that the L2 cache never holds a step's KV.
+그래프 리플레이); consecutive steps read different replicas of the KV pool, and
+the replicas together are larger than the L2 cache, so no step finds its KV
+in L2.
+
+The headline workload is the largest single-GPU one at the pages' f16
+precision: Qwen2.5-7B-shaped, B=128, 28/4 heads, contexts U[512, 4096], with
+the 128-token cache write fused into the step. The same line carries the
+other decode workloads (FP8 E4M3 cache, Qwen2.5-1.5B-shaped, and the skewed
+long-context batch at 512-token partitions and under the balanced plan), each
+with its own roofline, and the standalone cache write.
 
 Metric: algorithmic HBM bytes of the step (KV + Q + O + block tables +
 lengths for attention, plus the cache write's reads and writes) per second of
@@ -45,6 +53,10 @@ METRIC = "paged GQA decode attn: KV-read GB/s (% of B200 HBM peak), seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2 ** 20
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_attention_traffic.json")
+# the largest single-GPU decode workload at f16, and the others reported beside it (partition -1 is
+# the balanced plan, P > 0 fixed partitions of P tokens)
+HEADLINE = "qwen2.5-7b"
+SUBLINES = (("fp8-e4m3", -1), ("qwen2.5-1.5b", -1), ("skewed-split", 512), ("skewed-split", -1))
 
 
 # ------------------------------------------------------------------ byte model
@@ -347,7 +359,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="qwen2.5-1.5b", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition", type=int, default=-1,
                     help="split-KV plan: -1 the library's balanced plan (default), 0 single pass, "
@@ -362,9 +374,17 @@ def parse_args(argv=None):
                     help="skip timing the chunked prefill attention at the workload's head shape")
     ap.add_argument("--no-qkv", action="store_true",
                     help="skip timing the fused add + RMSNorm + QKV projection at the workload's shape")
+    ap.add_argument("--no-sublines", action="store_true",
+                    help="skip the other decode workloads (FP8, 1.5B, skewed at 512-token partitions and "
+                         "under the balanced plan) and the standalone cache write")
+    ap.add_argument("--sub-steps", type=int, default=200, help="timed steps of each other workload")
     ap.add_argument("--fp8-scales", default="tensor", choices=["tensor", "per-head"],
                     help="FP8 workloads: per-tensor host scales, or per-KV-head scales computed on the "
                          "device and passed to the device-scale entry points")
+    ap.add_argument("--kv-read-ratio", action="store_true",
+                    help="only compare the grouped decode kernel with per-query-head launches on the "
+                         "workload (one launch of each, then timed repeats): the KV bytes the grouping "
+                         "saves, for an ncu capture of dram__bytes_read")
     ap.add_argument("--cpu-baseline-s", type=float, default=10.0)
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args(argv)
@@ -404,6 +424,403 @@ def run_reference(args):
     return 0
 
 
+# A spin of about 0.5 ms queued in front of every timed region: the GPU is busy
+# while the host enqueues the timed graph replays, so the region measures the
+# steps on the device and not the host's submission latency.
+LEAD_IN_CYCLES = 1_000_000
+
+
+def lead_in(stream):
+    import torch
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(LEAD_IN_CYCLES)
+
+
+class StepBench:
+    """One decode workload resident on the device, and the library calls of its step.
+
+    The step is the whole hot path over the batch: this step's new K/V written at
+    position L_b - 1 of every sequence, then decode attention over the paged
+    contexts. With the balanced plan (partition -1) it is one fused launch
+    (paged_gqa_decode_step); with fixed partitions, or `unfused`, it is
+    paged_kv_cache_write followed by paged_gqa_decode_attention.
+
+    The KV pool is replicated R times and step i uses replica i % R, so that the
+    KV touched between two reads of one replica is at least 4x the L2 size; with
+    the overlap flag R >= 2, so that the launch before a step never writes the
+    pages that step reads before its grid-dependency wait (the flag's promise).
+    """
+
+    def __init__(self, w, device, stream, seed, partition, *, unfused=False, overlap=True,
+                 fp8_scales="tensor"):
+        import torch
+
+        import paged_kv_decode_gqa_b200 as pkv
+        self.torch, self.pkv = torch, pkv
+        self.w, self.device, self.stream, self.P = w, device, stream, partition
+        x = W.make_inputs(w, seed)
+        self.x = x
+        lens = x["context_lens"]
+        B, Hq, Hkv, D, bs = w.B, w.Hq, w.Hkv, w.head_dim, w.block_size
+        self.B = B
+        self.max_len = int(lens.max())
+        self.fp8 = fp8 = w.kv_dtype == "fp8"
+        self.attn_b, self.cw_b = step_bytes(w, lens, B)
+        self.step_b = self.attn_b + self.cw_b
+        self.fused = not unfused and partition == pkv.PKV_PARTITION_AUTO
+        self.flags = pkv.PKV_STEP_OVERLAP_PREVIOUS if (overlap and self.fused) else 0
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.t = t
+        self.q, self.bt, self.cl = t(x["q"]), t(x["block_tables"]), t(x["context_lens"])
+        self.k_new, self.v_new, self.slots = t(x["k_new"]), t(x["v_new"]), t(x["slot_mapping"])
+        self.ks, self.vs, self.scale = float(x["k_scale"]), float(x["v_scale"]), float(x["softmax_scale"])
+
+        self.touched = kv_bytes(lens, Hkv, D, 1 if fp8 else 2)
+        R = max(1, min(16, -(-4 * L2_BYTES // max(self.touched, 1))))
+        if self.flags:
+            R = max(R, 2)
+        self.R = R
+        k16, v16 = t(x["k_pool"]), t(x["v_pool"])
+        self.per_head = fp8 and fp8_scales == "per-head"
+        self.scales_kernel = None
+        if fp8:                                    # quantise the pool with the library's cache write
+            kq = torch.empty(k16.shape, dtype=torch.uint8, device=device)
+            vq = torch.empty_like(kq)
+            n_rows = w.num_blocks * bs
+            rows_k, rows_v = k16.view(n_rows, Hkv, D), v16.view(n_rows, Hkv, D)
+            all_slots = torch.arange(n_rows, dtype=torch.int64, device=device)
+            if self.per_head:
+                # per-KV-head scales computed on the device from the pool (its free rows are NaN
+                # and do not count); the scales kernel is timed over the K pool
+                self.ks_t = torch.empty(Hkv, dtype=torch.float32, device=device)
+                self.vs_t = torch.empty(Hkv, dtype=torch.float32, device=device)
+                for _ in range(3):
+                    pkv.paged_kv_fp8_scales(rows_k, self.ks_t, per_head=True, stream=stream)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                e0.record(stream)
+                for _ in range(reps):
+                    pkv.paged_kv_fp8_scales(rows_k, self.ks_t, per_head=True, stream=stream)
+                e1.record(stream)
+                pkv.paged_kv_fp8_scales(rows_v, self.vs_t, per_head=True, stream=stream)
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1000 / reps
+                nbytes = rows_k.numel() * 2
+                self.scales_kernel = {
+                    "input_bytes": nbytes, "us": us, "gbs": nbytes / us / 1e3,
+                    "what": "paged_kv_fp8_scales, per KV head, over the f16 K pool (memset + 2 launches)"}
+                pkv.paged_kv_cache_write_fp8_scaled(rows_k, rows_v, kq, vq, all_slots, self.ks_t, self.vs_t,
+                                                    stream=stream)
+            else:
+                pkv.paged_kv_cache_write(rows_k, rows_v, kq, vq, all_slots, kv_dtype="fp8", k_scale=self.ks,
+                                         v_scale=self.vs, stream=stream)
+            base_k, base_v = kq, vq
+            del k16, v16, rows_k, rows_v
+        else:
+            base_k, base_v = k16, v16
+        self.pools = [(base_k, base_v)] + [(base_k.clone(), base_v.clone()) for _ in range(R - 1)]
+        ws_n = pkv.paged_gqa_decode_workspace_size(B, Hq, Hkv, D, self.max_len, partition)
+        self.ws = torch.zeros(max(ws_n, 256), dtype=torch.uint8, device=device)
+        self.out = torch.empty((B, Hq, D), dtype=torch.float16, device=device)
+        torch.cuda.synchronize()
+
+    # ---- the library calls of one step: per-tensor scales or per-KV-head device scales ----
+    def write_call(self, kn, vn, kc, vc, sl):
+        if self.per_head:
+            self.pkv.paged_kv_cache_write_fp8_scaled(kn, vn, kc, vc, sl, self.ks_t, self.vs_t, stream=self.stream)
+        else:
+            self.pkv.paged_kv_cache_write(kn, vn, kc, vc, sl, kv_dtype=self.w.kv_dtype, k_scale=self.ks,
+                                          v_scale=self.vs, stream=self.stream)
+
+    def step_call(self, qq, kn, vn, kc, vc, bb, cc, flags):
+        if self.per_head:
+            self.pkv.paged_gqa_decode_step_fp8_scaled(self.out, qq, kn, vn, kc, vc, bb, cc, self.ks_t, self.vs_t,
+                                                      max_context_len=self.max_len, softmax_scale=self.scale,
+                                                      workspace=self.ws, flags=flags, stream=self.stream)
+        else:
+            self.pkv.paged_gqa_decode_step(self.out, qq, kn, vn, kc, vc, bb, cc, max_context_len=self.max_len,
+                                           softmax_scale=self.scale, kv_dtype=self.w.kv_dtype, k_scale=self.ks,
+                                           v_scale=self.vs, workspace=self.ws, flags=flags, stream=self.stream)
+
+    def attention_call(self, qq, kc, vc, bb, cc):
+        if self.per_head:
+            self.pkv.paged_gqa_decode_attention_fp8_scaled(self.out, qq, kc, vc, bb, cc, self.ks_t, self.vs_t,
+                                                           max_context_len=self.max_len, softmax_scale=self.scale,
+                                                           partition_tokens=self.P, workspace=self.ws,
+                                                           stream=self.stream)
+        else:
+            self.pkv.paged_gqa_decode_attention(self.out, qq, kc, vc, bb, cc, max_context_len=self.max_len,
+                                                softmax_scale=self.scale, kv_dtype=self.w.kv_dtype,
+                                                k_scale=self.ks, v_scale=self.vs, partition_tokens=self.P,
+                                                workspace=self.ws, stream=self.stream)
+
+    def step(self, i, events=None):
+        """Step i on pool replica i % R; `events` = (before, after) the attention launch."""
+        kc, vc = self.pools[i % self.R]
+        if self.fused:
+            self.step_call(self.q, self.k_new, self.v_new, kc, vc, self.bt, self.cl, self.flags)
+            return
+        self.write_call(self.k_new, self.v_new, kc, vc, self.slots)
+        if events:
+            events[0].record(self.stream)
+        self.attention_call(self.q, kc, vc, self.bt, self.cl)
+        if events:
+            events[1].record(self.stream)
+
+    @property
+    def launches_per_step(self):
+        return 1 if self.fused else 2
+
+    def warmup(self, n):
+        for i in range(n):
+            self.step(i)
+        self.torch.cuda.synchronize()
+
+    def time(self, K, graph_steps, world=1, sampler=None):
+        """Times exactly K steps replayed from CUDA graphs. Returns the device time of the region
+        (max over ranks), the attention kernel's mean launch duration and the host wall clock.
+
+        Graphs hold a multiple of R steps, so consecutive steps always use different replicas.
+        Fused: one launch per step and nothing between launches, so each launch overlaps the
+        previous one's tail (programmatic dependent launch); the kernel's average duration is the
+        region over K. Unfused: events around every attention launch give its own duration."""
+        torch = self.torch
+        S = max(1, min(graph_steps, K))
+        S = max(self.R, S - S % self.R)
+        chunks = [S] * (K // S) + ([K % S] if K % S else [])
+        graphs = {}
+        for n in sorted(set(chunks)):
+            evs = [] if self.fused else [(torch.cuda.Event(enable_timing=True, external=True),
+                                          torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                for i in range(n):
+                    self.step(i, evs[i] if evs else None)
+            graphs[n] = (g, evs)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, self.device)
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.start()
+        lead_in(self.stream)
+        wall0 = time.perf_counter()
+        start.record(self.stream)
+        for n in chunks:
+            graphs[n][0].replay()
+        end.record(self.stream)
+        torch.cuda.synchronize()
+        wall1 = time.perf_counter()
+        if sampler:
+            sampler.stop()
+        barrier(world, self.device)
+        elapsed_ms = start.elapsed_time(end)
+        if self.fused:
+            attn_ms = elapsed_ms / K
+        else:        # per-launch durations of the attention kernel in the last replay of each graph
+            d = [a.elapsed_time(b) for n in set(chunks) for a, b in graphs[n][1]]
+            attn_ms = sum(d) / len(d)
+        del graphs
+        return {"elapsed_ms": reduce_max(elapsed_ms, world, self.device), "attn_ms": attn_ms,
+                "wall": (wall0, wall1), "graph_steps": S, "replays": len(chunks)}
+
+    def e2e(self, n_steps, world=1):
+        """The same step through the public API on pinned host buffers: every step copies its
+        inputs host to device, runs, copies the output back and waits for it."""
+        torch = self.torch
+        x = self.x
+        h = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
+             for k in ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")}
+        d = {k: torch.empty(v.shape, dtype=v.dtype, device=self.device) for k, v in h.items()}
+        out_h = torch.empty(tuple(self.out.shape), dtype=torch.float16).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in h.values())
+        d2h = out_h.numel() * out_h.element_size()
+
+        def one(i):
+            for k in h:
+                d[k].copy_(h[k], non_blocking=True)
+            kc, vc = self.pools[i % self.R]
+            if self.fused:
+                self.step_call(d["q"], d["k_new"], d["v_new"], kc, vc, d["block_tables"], d["context_lens"], 0)
+            else:
+                self.write_call(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"])
+                self.attention_call(d["q"], kc, vc, d["block_tables"], d["context_lens"])
+            out_h.copy_(self.out, non_blocking=True)
+            self.stream.synchronize()
+
+        with torch.cuda.stream(self.stream):
+            for i in range(3):
+                one(i)
+            barrier(world, self.device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for i in range(n_steps):
+                one(i)
+            e1.record(self.stream)
+        torch.cuda.synchronize()
+        ms = reduce_max(e0.elapsed_time(e1), world, self.device)
+        return {"value": world * self.step_b * n_steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
+                "ms_per_step": ms / n_steps, "note": "eager calls, one host sync per step"}
+
+    def describe(self):
+        s = ("one fused launch (cache write + attention)" +
+             (", PKV_STEP_OVERLAP_PREVIOUS" if self.flags else "")) if self.fused \
+            else "cache write + attention launches"
+        return {"step": s,
+                "l2": f"inputs larger than L2: {self.R} KV pool replicas rotated, "
+                      f"{self.R * self.touched / 2**20:.0f} MiB touched per cycle"}
+
+
+def kernel_line(sb, timing, peak, peak_src):
+    """Roofline of the step's dominant kernel: algorithmic bytes per launch over its mean duration."""
+    kern_b = sb.step_b if sb.fused else sb.attn_b      # the fused launch also does the cache write
+    achieved = kern_b / (timing["attn_ms"] * 1e-3) / 1e9
+    return {"bound": "hbm",
+            "kernel": "decode_balanced_kernel (fused step)" if sb.fused else "decode attention",
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{peak_src} hbm_gbs", "traffic": recorded_traffic(sb.w.name, sb.P),
+            "algorithmic_bytes_per_launch": kern_b, "mean_launch_us": timing["attn_ms"] * 1e3}
+
+
+def time_subline(name, partition, device, stream, peak, peak_src, steps, seed, fp8_scales):
+    """One other decode workload: its own step, timed like the headline's, as a sub-object."""
+    import torch
+    w = W.WORKLOADS[name]
+    sb = StepBench(w, device, stream, seed, partition, fp8_scales=fp8_scales)
+    sb.warmup(5)
+    tm = sb.time(steps, 500)
+    roof = kernel_line(sb, tm, peak, peak_src)
+    res = {"workload": name, "partition_tokens": partition, **sb.describe(),
+           "steps": steps, "us_per_step": tm["elapsed_ms"] * 1e3 / steps,
+           "value": sb.step_b * steps / (tm["elapsed_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+           "seq_steps_per_s": w.B * steps / (tm["elapsed_ms"] * 1e-3),
+           "us": roof["mean_launch_us"], "achieved": roof["achieved"], "frac": roof["frac"],
+           "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"], "traffic": roof["traffic"],
+           "kernel": roof["kernel"], "gpu_launches": sb.launches_per_step * steps}
+    del sb
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_cache_write(w, device, stream, peak, seed=0, reps=200):
+    """paged_kv_cache_write alone at the workload's shape (one new token per sequence), from a
+    CUDA graph of `reps` launches that rotates over cache replicas larger than L2 in total."""
+    import torch
+
+    import paged_kv_decode_gqa_b200 as pkv
+    x = W.make_inputs(w, seed, poison=False)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    fp8 = w.kv_dtype == "fp8"
+    k_new, v_new, slots = t(x["k_new"]), t(x["v_new"]), t(x["slot_mapping"])
+    shape = x["k_pool"].shape
+    dt = torch.uint8 if fp8 else torch.float16
+    pool_bytes = 2 * int(np.prod(shape)) * (1 if fp8 else 2)
+    R = max(2, min(16, -(-2 * L2_BYTES // pool_bytes)))
+    pools = [(torch.zeros(shape, dtype=dt, device=device), torch.zeros(shape, dtype=dt, device=device))
+             for _ in range(R)]
+    call = lambda i: pkv.paged_kv_cache_write(k_new, v_new, pools[i % R][0], pools[i % R][1], slots,
+                                              kv_dtype=w.kv_dtype, k_scale=float(x["k_scale"]),
+                                              v_scale=float(x["v_scale"]), stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize()
+        n = max(R, reps - reps % R)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                call(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        lead_in(stream)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1000 / n
+    T = int((x["slot_mapping"] >= 0).sum())
+    nbytes = cache_write_bytes(T, w.Hkv, w.head_dim, 1 if fp8 else 2)
+    del g
+    return {"what": "paged_kv_cache_write (reshape_and_cache) alone", "workload": w.name, "T": T,
+            "Hkv": w.Hkv, "head_dim": w.head_dim, "kv_dtype": w.kv_dtype, "algorithmic_bytes": nbytes,
+            "us": us, "achieved": nbytes / us / 1e3, "peak": peak, "unit": "GB/s",
+            "frac": nbytes / us / 1e3 / peak, "bound": "hbm (launch-bound at this size)", "launches": n,
+            "l2": f"{R} cache replicas rotated; graph of {n} launches"}
+
+
+def run_kv_read_ratio(args):
+    """The grouped kernel against per-query-head launches on one workload: one launch of the
+    grouped attention (all G query heads of a KV head from one read of its K/V), then G launches
+    with Hq = Hkv, launch m serving query head m of every group, so every query head reads the
+    KV on its own. The first 1 + G decode launches of this process are exactly these, in this
+    order, for an ncu capture of dram__bytes_read.sum; timed repeats with L2 flushed follow."""
+    import torch
+
+    import paged_kv_decode_gqa_b200 as pkv
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w, args.seed)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    B, Hq, Hkv, D, G = w.B, w.Hq, w.Hkv, w.head_dim, w.group
+    if w.kv_dtype != "f16":
+        raise SystemExit("--kv-read-ratio takes an f16 workload")
+    k, v, bt, cl, q = t(x["k_pool"]), t(x["v_pool"]), t(x["block_tables"]), t(x["context_lens"]), t(x["q"])
+    max_len, scale = int(x["context_lens"].max()), float(x["softmax_scale"])
+    q_m = [q.view(B, Hkv, G, D)[:, :, m, :].contiguous() for m in range(G)]
+    out = torch.empty_like(q)
+    out_m = [torch.empty_like(qm) for qm in q_m]
+    P = pkv.PKV_PARTITION_AUTO
+    ws = torch.zeros(max(pkv.paged_gqa_decode_workspace_size(B, Hq, Hkv, D, max_len, P), 256),
+                     dtype=torch.uint8, device=device)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+
+    def grouped():
+        pkv.paged_gqa_decode_attention(out, q, k, v, bt, cl, max_context_len=max_len, softmax_scale=scale,
+                                       partition_tokens=P, workspace=ws, stream=stream)
+
+    def per_head(m):
+        pkv.paged_gqa_decode_attention(out_m[m], q_m[m], k, v, bt, cl, max_context_len=max_len,
+                                       softmax_scale=scale, partition_tokens=P, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        grouped()
+        for m in range(G):
+            per_head(m)
+        torch.cuda.synchronize()
+        ref = out.view(B, Hkv, G, D)
+        same = all(torch.equal(out_m[m], ref[:, :, m, :]) for m in range(G))
+        max_diff = max(float((out_m[m].float() - ref[:, :, m, :].float()).abs().max()) for m in range(G))
+
+        def timed(fn, reps=20):
+            ms = []
+            for _ in range(reps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ms.append(e0.elapsed_time(e1))
+            return statistics.median(ms) * 1e3
+
+        us_grouped = timed(grouped)
+        us_per_head = timed(lambda: [per_head(m) for m in range(G)])
+    kv = kv_bytes(x["context_lens"], Hkv, D, 2)
+    print(json.dumps({
+        "what": "grouped decode attention vs per-query-head launches (Hq = Hkv, one launch per group member)",
+        "workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "G": G,
+        "kv_bytes_grouped": kv, "kv_bytes_per_query_head": G * kv,
+        "outputs_bitwise_equal": same, "max_abs_diff": max_diff,
+        "us_grouped": us_grouped, "us_per_query_head_total": us_per_head,
+        "time_ratio": us_per_head / us_grouped,
+        "timing": "median of 20, L2 flushed (256 MiB write) before each"}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -415,243 +832,66 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    import paged_kv_decode_gqa_b200 as pkv
 
     w = W.WORKLOADS[args.workload]
-    x = W.make_inputs(w, W.shard_seed(args.seed, rank))
-    lens = x["context_lens"]
-    B, Hq, Hkv, D, bs = w.B, w.Hq, w.Hkv, w.head_dim, w.block_size
-    max_len = int(lens.max())
-    fp8 = w.kv_dtype == "fp8"
-    P = args.partition
-    attn_b, cw_b = step_bytes(w, lens, B)
-    step_b = attn_b + cw_b
-
     stream = torch.cuda.Stream(device)
     torch.cuda.set_stream(stream)
-    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-    q, bt, cl = t(x["q"]), t(x["block_tables"]), t(x["context_lens"])
-    k_new, v_new, slots = t(x["k_new"]), t(x["v_new"]), t(x["slot_mapping"])
-    ks, vs, scale = float(x["k_scale"]), float(x["v_scale"]), float(x["softmax_scale"])
-
-    # KV pool replicas: enough that the KV touched between two reads of a replica exceeds 4x L2.
-    touched = kv_bytes(lens, Hkv, D, 1 if fp8 else 2)
-    R = max(1, min(16, -(-4 * L2_BYTES // max(touched, 1))))
-    k16, v16 = t(x["k_pool"]), t(x["v_pool"])
-    per_head = fp8 and args.fp8_scales == "per-head"
-    scales_kernel = None
-    if fp8:                                        # quantise the pool with the library's cache write
-        kq = torch.empty(k16.shape, dtype=torch.uint8, device=device)
-        vq = torch.empty_like(kq)
-        n_rows = w.num_blocks * bs
-        rows_k, rows_v = k16.view(n_rows, Hkv, D), v16.view(n_rows, Hkv, D)
-        all_slots = torch.arange(n_rows, dtype=torch.int64, device=device)
-        if per_head:
-            # per-KV-head scales computed on the device from the pool (its free rows are NaN and
-            # do not count); the scales kernel is timed over the K pool
-            ks_t = torch.empty(Hkv, dtype=torch.float32, device=device)
-            vs_t = torch.empty(Hkv, dtype=torch.float32, device=device)
-            for _ in range(3):
-                pkv.paged_kv_fp8_scales(rows_k, ks_t, per_head=True, stream=stream)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 10
-            e0.record(stream)
-            for _ in range(reps):
-                pkv.paged_kv_fp8_scales(rows_k, ks_t, per_head=True, stream=stream)
-            e1.record(stream)
-            pkv.paged_kv_fp8_scales(rows_v, vs_t, per_head=True, stream=stream)
-            torch.cuda.synchronize()
-            us = e0.elapsed_time(e1) * 1000 / reps
-            nbytes = rows_k.numel() * 2
-            scales_kernel = {"input_bytes": nbytes, "us": us, "gbs": nbytes / us / 1e3,
-                             "what": "paged_kv_fp8_scales, per KV head, over the f16 K pool (memset + 2 launches)"}
-            pkv.paged_kv_cache_write_fp8_scaled(rows_k, rows_v, kq, vq, all_slots, ks_t, vs_t, stream=stream)
-        else:
-            pkv.paged_kv_cache_write(rows_k, rows_v, kq, vq, all_slots, kv_dtype="fp8", k_scale=ks, v_scale=vs)
-        base_k, base_v = kq, vq
-        del k16, v16, rows_k, rows_v
-    else:
-        base_k, base_v = k16, v16
-    pools = [(base_k, base_v)] + [(base_k.clone(), base_v.clone()) for _ in range(R - 1)]
-    ws_n = pkv.paged_gqa_decode_workspace_size(B, Hq, Hkv, D, max_len, P)
-    ws = torch.zeros(max(ws_n, 256), dtype=torch.uint8, device=device)
-    out = torch.empty((B, Hq, D), dtype=torch.float16, device=device)
-
-    fused = not args.unfused and P == pkv.PKV_PARTITION_AUTO
-    step_flags = 0 if args.no_overlap else pkv.PKV_STEP_OVERLAP_PREVIOUS
-
-    # the library calls of one step, per-tensor scales or per-KV-head device scales
-    def write_call(kn, vn, kc, vc, sl):
-        if per_head:
-            pkv.paged_kv_cache_write_fp8_scaled(kn, vn, kc, vc, sl, ks_t, vs_t, stream=stream)
-        else:
-            pkv.paged_kv_cache_write(kn, vn, kc, vc, sl, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                     stream=stream)
-
-    def step_call(qq, kn, vn, kc, vc, bb, cc, flags):
-        if per_head:
-            pkv.paged_gqa_decode_step_fp8_scaled(out, qq, kn, vn, kc, vc, bb, cc, ks_t, vs_t,
-                                                 max_context_len=max_len, softmax_scale=scale,
-                                                 workspace=ws, flags=flags, stream=stream)
-        else:
-            pkv.paged_gqa_decode_step(out, qq, kn, vn, kc, vc, bb, cc, max_context_len=max_len,
-                                      softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks, v_scale=vs,
-                                      workspace=ws, flags=flags, stream=stream)
-
-    def attention_call(qq, kc, vc, bb, cc):
-        if per_head:
-            pkv.paged_gqa_decode_attention_fp8_scaled(out, qq, kc, vc, bb, cc, ks_t, vs_t,
-                                                      max_context_len=max_len, softmax_scale=scale,
-                                                      partition_tokens=P, workspace=ws, stream=stream)
-        else:
-            pkv.paged_gqa_decode_attention(out, qq, kc, vc, bb, cc, max_context_len=max_len,
-                                           softmax_scale=scale, kv_dtype=w.kv_dtype, k_scale=ks,
-                                           v_scale=vs, partition_tokens=P, workspace=ws, stream=stream)
-
-    def cache_write(i):
-        if fused:                                  # the step kernel writes the new tokens itself
-            return
-        kc, vc = pools[i % R]
-        write_call(k_new, v_new, kc, vc, slots)
-
-    def attention(i):
-        kc, vc = pools[i % R]
-        if fused:
-            # consecutive steps read different pool replicas, so no launch writes
-            # the pages the next one reads: the overlap promise holds
-            step_call(q, k_new, v_new, kc, vc, bt, cl, step_flags)
-        else:
-            attention_call(q, kc, vc, bt, cl)
-
-    # ---- warm-up: W eager steps (also sets kernel attributes and TMA maps) ----
-    for i in range(args.warmup):
-        cache_write(i)
-        attention(i)
-    torch.cuda.synchronize()
-
-    # ---- capture the timed steps as CUDA graphs with events around each attention launch ----
+    sb = StepBench(w, device, stream, W.shard_seed(args.seed, rank), args.partition, unfused=args.unfused,
+                   overlap=not args.no_overlap, fp8_scales=args.fp8_scales)
+    B = w.B
     K = args.steps
-    S = max(1, min(args.graph_steps, K))
-    chunks = [S] * (K // S) + ([K % S] if K % S else [])
-    graphs, ev_pairs = {}, []
-    # Fused: one launch per step and nothing between launches, so that each
-    # launch overlaps the previous one's tail (programmatic dependent launch);
-    # its average duration is the timed region over K. Unfused: events around
-    # every attention launch give that kernel's own duration.
-    for n in sorted(set(chunks)):
-        evs = [] if fused else [(torch.cuda.Event(enable_timing=True, external=True),
-                                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                cache_write(i)
-                if evs:
-                    evs[i][0].record(stream)
-                attention(i)
-                if evs:
-                    evs[i][1].record(stream)
-        graphs[n] = (g, evs)
-    torch.cuda.synchronize()
 
-    sampler = ClockSampler(torch.cuda.current_device()).start()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    attn_ms = []
-    barrier(world, device)
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    start.record(stream)
-    for n in chunks:
-        graphs[n][0].replay()
-    end.record(stream)
-    torch.cuda.synchronize()
-    wall1 = time.perf_counter()
-    barrier(world, device)
-    sampler.stop()
-    elapsed_ms = start.elapsed_time(end)
-    if fused:
-        attn_ms = [elapsed_ms / K]
-    else:        # per-launch durations of the attention kernel in the last replay of each graph
-        for n in set(chunks):
-            attn_ms += [a.elapsed_time(b) for a, b in graphs[n][1]]
-    elapsed_max = reduce_max(elapsed_ms, world, device)
-    launches = (1 if fused else 2) * K
-
-    # ---- e2e: the public API on host buffers, copies in the timed region ----
-    e2e = None
-    if not args.no_e2e:
-        h = {k: torch.from_numpy(np.ascontiguousarray(x[k])).pin_memory()
-             for k in ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")}
-        d = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in h.items()}
-        out_h = torch.empty((B, Hq, D), dtype=torch.float16).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in h.values())
-        d2h = out_h.numel() * out_h.element_size()
-        n_e2e = max(3, min(K, 200))
-
-        def e2e_step(i):
-            for k in h:
-                d[k].copy_(h[k], non_blocking=True)
-            kc, vc = pools[i % R]
-            if fused:
-                step_call(d["q"], d["k_new"], d["v_new"], kc, vc, d["block_tables"], d["context_lens"], 0)
-            else:
-                write_call(d["k_new"], d["v_new"], kc, vc, d["slot_mapping"])
-                attention_call(d["q"], kc, vc, d["block_tables"], d["context_lens"])
-            out_h.copy_(out, non_blocking=True)
-            stream.synchronize()
-
-        for i in range(3):
-            e2e_step(i)
-        barrier(world, device)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(n_e2e):
-            e2e_step(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = reduce_max(e0.elapsed_time(e1), world, device)
-        e2e = {"value": world * step_b * n_e2e / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "ms_per_step": e2e_ms / n_e2e, "note": "eager calls, one host sync per step"}
+    # ---- warm-up: W eager steps (also sets kernel attributes and TMA maps), then K timed steps ----
+    sb.warmup(args.warmup)
+    sampler = ClockSampler(torch.cuda.current_device())
+    tm = sb.time(K, args.graph_steps, world, sampler)
+    elapsed_max = tm["elapsed_ms"]
+    e2e = None if args.no_e2e else sb.e2e(max(3, min(K, 200)), world)
 
     if rank == 0:
         peaks, peak_src = measured_peaks()
         peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-        mean_attn_ms = sum(attn_ms) / len(attn_ms)
-        kern_b = step_b if fused else attn_b          # the fused launch also does the cache write
-        achieved = kern_b / (mean_attn_ms * 1e-3) / 1e9
-        traffic = recorded_traffic(w.name, P)
-        value = whole_job_gbs(world, step_b, K, elapsed_max)
+        value = whole_job_gbs(world, sb.step_b, K, elapsed_max)
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_max / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16" if not fp8 else "fp8-e4m3 KV, f16 q/out",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16" if not sb.fp8 else "fp8-e4m3 KV, f16 q/out",
             "data": "synthetic",
             "seq_steps_per_s": world * B * K / (elapsed_max * 1e-3),
             "pct_of_hbm_peak": 100.0 * value / peak,
-            "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "head_dim": D,
-                       "block_size": bs, "kv_dtype": w.kv_dtype, "context_lens": list(w.ctx),
-                       **({"fp8_scales": "per KV head, computed on the device"} if per_head else {}),
-                       "partition_tokens": P, "parallelism": f"dp{world} (independent batches)",
-                       "l2": f"inputs larger than L2: {R} KV pool replicas rotated, "
-                             f"{R * touched / 2**20:.0f} MiB touched per cycle",
-                       "timing": f"{len(chunks)} CUDA graph replays of <= {S} steps",
-                       "step": ("one fused launch (cache write + attention)" +
-                                ("" if args.no_overlap else ", PKV_STEP_OVERLAP_PREVIOUS"))
-                               if fused else "cache write + attention launches"},
-            "roofline": {"bound": "hbm",
-                         "kernel": "decode_balanced_kernel (fused step)" if fused else "decode attention",
-                         "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
-                         "traffic": traffic, "algorithmic_bytes_per_launch": kern_b,
-                         "mean_launch_us": mean_attn_ms * 1e3},
-            "gpu_launches": launches,
-            "clocks": sampler.summary(wall0, wall1),
+            "config": {"workload": w.name, "B": B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.head_dim,
+                       "block_size": w.block_size, "kv_dtype": w.kv_dtype, "context_lens": list(w.ctx),
+                       **({"fp8_scales": "per KV head, computed on the device"} if sb.per_head else {}),
+                       "partition_tokens": args.partition, "parallelism": f"dp{world} (independent batches)",
+                       **sb.describe(),
+                       "timing": f"{tm['replays']} CUDA graph replays of <= {tm['graph_steps']} steps after a "
+                                 "0.5 ms lead-in spin, CUDA events on the launching stream"},
+            "roofline": kernel_line(sb, tm, peak, peak_src),
+            "gpu_launches": sb.launches_per_step * K,
+            "clocks": sampler.summary(*tm["wall"]),
         }
-        if scales_kernel:
-            line["fp8_scales_kernel"] = scales_kernel
-        # side measurements of the other kernels: a failure is reported in its key, and the
-        # step's line is still printed
+        if sb.scales_kernel:
+            line["fp8_scales_kernel"] = sb.scales_kernel
+        if e2e:
+            line["e2e"] = e2e
+        del sb
+        torch.cuda.empty_cache()
+        # side measurements: a failure is reported in its key, and the step's line is still printed
         side = []
+        if not args.no_sublines and world == 1:
+            subs = {}
+            for name, P in SUBLINES:
+                if name == w.name and P == args.partition:
+                    continue
+                key = f"{name}/{'auto' if P == -1 else f'P{P}'}"
+                try:
+                    subs[key] = time_subline(name, P, device, stream, peak, peak_src, args.sub_steps, args.seed,
+                                             args.fp8_scales)
+                except Exception as exc:  # noqa: BLE001 -- reported, never silent
+                    subs[key] = {"error": f"{type(exc).__name__}: {exc}"}
+            line["workloads"] = subs
+            side.append(("cache_write_kernel", lambda: time_cache_write(W.WORKLOADS[HEADLINE], device, stream,
+                                                                        peak, args.seed)))
         if not args.no_qkv:
             side.append(("qkv_kernel", lambda: time_qkv_projection(w, device, stream, peak, args.seed)))
         if not args.no_prefill:
@@ -662,15 +902,14 @@ def run_ours(args):
                 line[key] = measure()
             except Exception as exc:  # noqa: BLE001 -- reported, never silent
                 line[key] = {"error": f"{type(exc).__name__}: {exc}"}
-        if e2e:
-            line["e2e"] = e2e
         if world == 1 and args.cpu_baseline_s > 0:
+            x = W.make_inputs(w, W.shard_seed(args.seed, rank))
             reps, secs, cores = time_oracle(w, x, args.cpu_baseline_s)
+            attn_b, cw_b = step_bytes(w, x["context_lens"], B)
             line["cpu_baseline"] = {
-                "value": step_b * reps / secs / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "value": (attn_b + cw_b) * reps / secs / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
                 "sample": f"{reps} whole steps of {w.name} (all {B} sequences), {secs:.1f} s"}
         print(json.dumps(line), flush=True)
-    del graphs
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
@@ -682,6 +921,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.kv_read_ratio:
+        return run_kv_read_ratio(args)
     return run_ours(args)
 
 
