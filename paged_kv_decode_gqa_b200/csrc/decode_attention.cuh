@@ -189,9 +189,8 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
     const float out_scale = p.v_scales ? head_scale(p.v_scales, p.scales_per_head, g) : p.out_scale;
     if (p.k_scales && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
         check_scales(p.k_scales, p.v_scales, p.scales_per_head ? p.Hkv : 1, 0, 1);
-    uint32_t qf[8][2];
-    load_q_fragments<kFp8>(
-        qf, r < G ? p.q + ((int64_t)b * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, c);
+    QOperand<kFp8> qf;
+    load_q_fragments(qf, r < G ? p.q + ((int64_t)b * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, lane);
     WarpState st;
     st.reset();
 

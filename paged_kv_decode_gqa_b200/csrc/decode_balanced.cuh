@@ -17,7 +17,8 @@
 //  * A worker's range cuts (sequence, KV head) segments into pieces. A piece
 //    that is a whole segment writes the output directly. Otherwise the piece
 //    writes (m, l, O/l) to the workspace in the warp's fragment order
-//    (coalesced 16-byte stores) and joins a merge tree of fan-in 32: the last
+//    (fragment i of all 32 lanes in one 512-byte run, so every store and load
+//    of an item is fully coalesced) and joins a merge tree of fan-in 32: the last
 //    of each group of 32 items to finish (an atomic ticket) merges the group
 //    by the log-sum-exp rule into the slot of the group's first piece, which
 //    is an item of the next level; the merge that leaves one item writes the
@@ -35,7 +36,7 @@ struct BalancedParams {
     const __half* q;              // [B, Hq, D]
     const int32_t* block_tables;  // [B, max_blocks_per_seq]
     const int32_t* context_lens;  // [B]
-    float4* ws_o;                 // [2 * workers][32 lanes][8 float4]   piece outputs O/l
+    float4* ws_o;                 // [2 * workers][8][32 lanes] float4   piece outputs O/l
     float4* ws_ml;                // [2 * workers][4] (m, l) pairs of heads 2c, 2c+1
     unsigned int* ws_count;       // [kMergeLevels][2 * workers] tickets of the merge tree
     // fused decode step only: this step's token of every sequence, written to
@@ -60,8 +61,16 @@ struct BalancedParams {
     uint64_t wait_limit_ns;
 };
 
-constexpr int kMergeFloats = 32 * 8 + 16;     // per warp: weights of 32 items x 8 heads, M, L
-constexpr int kMergeLevels = 4;               // fan-in 32: up to 32^4 pieces per segment
+// Fan-in of the merge tree (at most 32, one item per lane when merging);
+// kMergeLevels levels cover every worker of the largest grid.
+#ifndef PKV_MERGE_FAN
+#define PKV_MERGE_FAN 32
+#endif
+constexpr int kMergeFan = PKV_MERGE_FAN;
+static_assert(kMergeFan >= 2 && kMergeFan <= 32, "merge fan-in");
+constexpr int kMergeFloats = 32 * 8 + 16;     // per warp: weights of up to 32 items x 8 heads, M, L
+constexpr int merge_levels(int fan) { int l = 1, n = fan; while (n < 4096) { n *= fan; ++l; } return l; }
+constexpr int kMergeLevels = merge_levels(kMergeFan);   // fan^levels >= 4096 pieces per segment
 
 template <bool kFp8, int kWarps, int kStages>
 struct BalancedShape {
@@ -107,6 +116,13 @@ __device__ __forceinline__ uint32_t quantize4_e4m3(uint2 x, float scale) {
     }
     return out;
 }
+
+// Merges at the end of a worker's range stage the items' values in the
+// worker's free ring by cp.async (1) or load them into registers like merges
+// mid-range (0); a tuning switch.
+#ifndef PKV_MERGE_STAGED
+#define PKV_MERGE_STAGED 0
+#endif
 
 // Two consecutive pages of one segment per online-softmax step (when the
 // segment has them in the worker's range): two independent logit chains and
@@ -285,8 +301,8 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     auto q_row = [&](int bb, int gg) -> const __half* {
         return r < G ? p.q + ((int64_t)bb * p.Hq + (int64_t)gg * G + r) * kHeadDim : nullptr;
     };
-    uint32_t qf[8][2];
-    load_q_fragments<kFp8>(qf, q_row(b, g), c);
+    QOperand<kFp8> qf;
+    load_q_fragments(qf, q_row(b, g), lane);
     // scales of the current segment's KV head (device scales are read after the wait)
     float sl = p.logit_scale_log2, out_scale = p.out_scale, k_quant = p.k_scale, v_quant = p.v_scale;
     auto set_head_scales = [&](int gg) {
@@ -321,15 +337,16 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
     };
     // (m, l, O/l) of one partial result, in fragment order, at workspace slot sl.
     auto store_item = [&](int sl, const float (&v)[8][4], float m0, float l0, float m1, float l1) {
-        float4* dst = p.ws_o + ((int64_t)sl * 32 + lane) * 8;
+        float4* dst = p.ws_o + (int64_t)sl * 256 + lane;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
+        for (int i = 0; i < 8; ++i) dst[32 * i] = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
         if (r == 0) p.ws_ml[(int64_t)sl * 4 + c] = make_float4(m0, l0, m1, l1);
     };
     float* wts = merge_scratch + warp * kMergeFloats;     // [32 items][8 heads] + M[8] + L[8]
 
-    // Finishes the piece of segment (b, g) whose last page is j_last.
-    auto finish_piece = [&](int j_last) {
+    // Finishes the piece of segment (b, g) whose last page is j_last. `at_end`:
+    // the worker's range ends here, so its ring is free to stage merge loads.
+    auto finish_piece = [&](int j_last, bool at_end) {
         st.reduce_l();
         if (piece_j0 == 0 && j_last == nb - 1) {          // the whole segment: write it
             write_out(st.o, out_scale / st.l0, out_scale / st.l1);
@@ -359,7 +376,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         int item = worker - k_first, n_items = k_last - k_first + 1, span = 1;
         store_item(slot_of_piece(item), v, m0, l0, m1, l1);
         for (int lvl = 0;; ++lvl) {
-            const int first = item & ~31, last = min(first + 32, n_items) - 1;
+            const int first = item - item % kMergeFan, last = min(first + kMergeFan, n_items) - 1;
             const int cslot = slot_of_piece(first * span);
             unsigned int* cnt = p.ws_count + (int64_t)lvl * 2 * W_total + cslot;
             // The warp barrier orders every lane's stores before lane 0's
@@ -370,23 +387,42 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             prev = __shfl_sync(0xffffffffu, prev, 0);
             if (prev != (unsigned int)(last - first)) return;   // another item merges the group
             // ---- merge items first..last ----
-            // (m, l) lane-parallel and the first two items' values are loaded
-            // together; later values are double-buffered two items at a time.
+            // (m, l) are loaded lane-parallel. The items' values come either
+            // staged in the worker's free ring (at the end of its range: up to
+            // the ring's size in 4 KiB items per round trip, by cp.async) or,
+            // mid-range (rare), through registers two items at a time.
             const int n_it = last - first + 1;
             const int my_slot = lane < n_it ? slot_of_piece((first + lane) * span) : 0;
+            constexpr int kBatch = kStages * S::kSlotBytes / 4096;        // items per staged round trip
+            const uint32_t stage = k_tile(0);
+            auto fetch = [&](int b0) {
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    if (b0 + u < n_it) {
+                        const int sl = __shfl_sync(0xffffffffu, my_slot, b0 + u);
+                        const float4* src = p.ws_o + (int64_t)sl * 256 + lane;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) cp_async16(stage + u * 4096 + lane * 128 + 16 * i, src + 32 * i);
+                    }
+                }
+                cp_async_commit();
+            };
             auto load_vals = [&](float4 (&dst)[2][8], int t) {
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     if (t + u < n_it) {
                         const int sl = __shfl_sync(0xffffffffu, my_slot, t + u);
-                        const float4* src = p.ws_o + ((int64_t)sl * 32 + lane) * 8;
+                        const float4* src = p.ws_o + (int64_t)sl * 256 + lane;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) dst[u][i] = __ldcg(src + i);
+                        for (int i = 0; i < 8; ++i) dst[u][i] = __ldcg(src + 32 * i);
                     }
                 }
             };
-            float4 va[2][8], vb[2][8];
-            load_vals(va, 0);
+            constexpr int kPairs = kFp8 ? 1 : 2;       // register buffers of two items (FP8: register-bound)
+            float4 va[kPairs][2][8];
+            const bool staged = PKV_MERGE_STAGED && at_end;
+            if (staged) fetch(0);
+            else load_vals(va[0], 0);
             float mm[8], ll[8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -413,30 +449,55 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
             float acc[8][4];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-            auto consume = [&](const float4 (&vals)[2][8], int t) {
+            auto add_item = [&](const float4 (&v)[8], int t) {
+                const float w0 = wts[t * 8 + 2 * c], w1 = wts[t * 8 + 2 * c + 1];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (t + u < n_it) {
-                        const float w0 = wts[(t + u) * 8 + 2 * c], w1 = wts[(t + u) * 8 + 2 * c + 1];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            acc[i][0] += w0 * vals[u][i].x; acc[i][1] += w1 * vals[u][i].y;
-                            acc[i][2] += w0 * vals[u][i].z; acc[i][3] += w1 * vals[u][i].w;
-                        }
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    acc[i][0] += w0 * v[i].x; acc[i][1] += w1 * v[i].y;
+                    acc[i][2] += w0 * v[i].z; acc[i][3] += w1 * v[i].w;
                 }
             };
-            for (int t0 = 0; t0 < n_it; t0 += 4) {
-                if (t0 + 2 < n_it) load_vals(vb, t0 + 2);
-                consume(va, t0);
-                if (t0 + 4 < n_it) load_vals(va, t0 + 4);
-                if (t0 + 2 < n_it) consume(vb, t0 + 2);
+            if (staged) {
+                for (int b0 = 0; b0 < n_it; b0 += kBatch) {
+                    cp_async_wait_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        if (b0 + u < n_it) {
+                            float4 v[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const uint4 raw = lds128(stage + u * 4096 + lane * 128 + 16 * i);
+                                v[i] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y),
+                                                   __uint_as_float(raw.z), __uint_as_float(raw.w));
+                            }
+                            add_item(v, b0 + u);
+                        }
+                    }
+                    __syncwarp();
+                    if (b0 + kBatch < n_it) fetch(b0 + kBatch);
+                }
+            } else {
+                // kPairs buffers: the loads of the next pairs are in flight while one is added
+#pragma unroll 1
+                for (int t0 = 0; t0 < n_it; t0 += 2 * kPairs) {
+#pragma unroll
+                    for (int k = 1; k < kPairs; ++k)
+                        if (t0 + 2 * k < n_it) load_vals(va[k], t0 + 2 * k);
+#pragma unroll
+                    for (int k = 0; k < kPairs; ++k) {
+#pragma unroll
+                        for (int u = 0; u < 2; ++u)
+                            if (t0 + 2 * k + u < n_it) add_item(va[k][u], t0 + 2 * k + u);
+                        if (k == 0 && t0 + 2 * kPairs < n_it) load_vals(va[0], t0 + 2 * kPairs);
+                    }
+                }
             }
             m0 = wts[256 + 2 * c]; m1 = wts[256 + 2 * c + 1];
             l0 = wts[264 + 2 * c]; l1 = wts[264 + 2 * c + 1];
             __syncwarp();
             if (lane == 0) *cnt = 0u;                          // ready for the next call
-            const int n_next = (n_items + 31) / 32;
+            const int n_next = (n_items + kMergeFan - 1) / kMergeFan;
             if (n_next == 1) {
                 write_out(acc, out_scale, out_scale);
                 return;
@@ -446,9 +507,9 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
                 v[i][0] = acc[i][0]; v[i][1] = acc[i][1]; v[i][2] = acc[i][2]; v[i][3] = acc[i][3];
             }
             store_item(cslot, v, m0, l0, m1, l1);              // the group is one item of level + 1
-            item = first / 32;
+            item = first / kMergeFan;
             n_items = n_next;
-            span *= 32;
+            span *= kMergeFan;
         }
     };
 
@@ -533,7 +594,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
         // advance the cursor; a segment boundary (or the range end) closes the piece
         const bool seg_end = j == nb - 1;
         if (seg_end || t == n - 1) {
-            finish_piece(j);
+            finish_piece(j, t == n - 1);
             if (t == n - 1) break;
             first_piece = false;
             st.reset();
@@ -544,7 +605,7 @@ decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
                     do { ++b; } while (units_of(b) == 0);
                     nb = units_of(b);
                 }
-                load_q_fragments<kFp8>(qf, q_row(b, g), c);
+                load_q_fragments(qf, q_row(b, g), lane);
                 set_head_scales(g);
             }
             piece_j0 = j;

@@ -51,19 +51,28 @@ __device__ __forceinline__ int out_channel_lo(int r, int i) { return kFp8 ? 16 *
 template <bool kFp8>
 __device__ __forceinline__ int out_channel_hi(int r, int i) { return kFp8 ? 16 * r + 2 * i + 1 : 16 * i + r + 8; }
 
-// Q^T as the B operand for the query head of row r (16 channels per k-step);
-// `qrow` is that head's 128 f16 channels, or nullptr for a padding head.
+// Q^T as the B operand of the logits (mma m16n8k16), for the query head of
+// row r (lane (r, c) = (lane / 4, lane % 4)); `qrow` is that head's 128 f16
+// channels, or nullptr for a padding head. The contraction may take the
+// channels in any order as long as K and Q agree:
+//  * f16 cache: channels 16j+2c(+1) and 16j+8+2c(+1) of k-step j;
+//  * FP8 cache: channels 16j+4c(+1) and 16j+4c+2(+1), matching the four E4M3
+//    codes per lane that ldmatrix delivers from the byte tile.
 template <bool kFp8>
-__device__ __forceinline__ void load_q_fragments(uint32_t (&qf)[8][2], const __half* qrow, int c) {
+struct QOperand {
+    uint32_t f[8][2];
+};
+
+template <bool kFp8>
+__device__ __forceinline__ void load_q_fragments(QOperand<kFp8>& q, const __half* qrow, int lane) {
+    const int c = lane & 3;
     const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        // f16 cache: channels 16j+2c(+1) and 16j+8+2c(+1);
-        // FP8 cache: channels 16j+4c(+1) and 16j+4c+2(+1), matching the byte tile fragments.
         const int d0 = kFp8 ? 16 * j + 4 * c : 16 * j + 2 * c;
         const int d1 = kFp8 ? d0 + 2 : d0 + 8;
-        qf[j][0] = qrow ? __ldg(q32 + d0 / 2) : 0u;
-        qf[j][1] = qrow ? __ldg(q32 + d1 / 2) : 0u;
+        q.f[j][0] = qrow ? __ldg(q32 + d0 / 2) : 0u;
+        q.f[j][1] = qrow ? __ldg(q32 + d1 / 2) : 0u;
     }
 }
 
@@ -72,7 +81,7 @@ __device__ __forceinline__ void load_q_fragments(uint32_t (&qf)[8][2], const __h
 // r (x[0], x[1]) and r + 8 (x[2], x[3]) of heads 2c, 2c + 1. K tile at shared
 // address kt (f16: two 2 KiB boxes of 64 channels each; FP8: one 2 KiB box).
 template <bool kFp8>
-__device__ __forceinline__ void page_logits(float (&x)[4], uint32_t kt, int valid, const uint32_t (&qf)[8][2],
+__device__ __forceinline__ void page_logits(float (&x)[4], uint32_t kt, int valid, const QOperand<kFp8>& qf,
                                             float sl, int lane) {
     const int r = lane >> 2;
     // Two independent accumulators (even and odd k-steps) halve the chain of
@@ -86,7 +95,7 @@ __device__ __forceinline__ void page_logits(float (&x)[4], uint32_t kt, int vali
             const uint32_t addr = kt + (kk >> 2) * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
-            mma_16816(sacc[kk & 1], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+            mma_16816(sacc[kk & 1], a0, a1, a2, a3, qf.f[kk][0], qf.f[kk][1]);
         }
     } else {
 #pragma unroll
@@ -95,12 +104,13 @@ __device__ __forceinline__ void page_logits(float (&x)[4], uint32_t kt, int vali
             const uint32_t addr = kt + row * 128 + ((chunk ^ (row & 7)) << 4);
             uint32_t r0, r1, r2, r3;            // 4 codes each: channels 16*chunk + 4c .. +3
             ldsm_x4(addr, r0, r1, r2, r3);
-            mma_16816(sacc[0], e4m3x2_to_half2(r0), e4m3x2_to_half2(r1),
-                      e4m3x2_to_half2(r0 >> 16), e4m3x2_to_half2(r1 >> 16),
-                      qf[2 * J][0], qf[2 * J][1]);
-            mma_16816(sacc[1], e4m3x2_to_half2(r2), e4m3x2_to_half2(r3),
-                      e4m3x2_to_half2(r2 >> 16), e4m3x2_to_half2(r3 >> 16),
-                      qf[2 * J + 1][0], qf[2 * J + 1][1]);
+            uint32_t h0l, h0h, h1l, h1h, h2l, h2h, h3l, h3h;
+            e4m3x4_to_half2x2(r0, h0l, h0h);
+            e4m3x4_to_half2x2(r1, h1l, h1h);
+            e4m3x4_to_half2x2(r2, h2l, h2h);
+            e4m3x4_to_half2x2(r3, h3l, h3h);
+            mma_16816(sacc[0], h0l, h1l, h0h, h1h, qf.f[2 * J][0], qf.f[2 * J][1]);
+            mma_16816(sacc[1], h2l, h3l, h2h, h3h, qf.f[2 * J + 1][0], qf.f[2 * J + 1][1]);
         }
     }
 #pragma unroll
@@ -153,8 +163,10 @@ __device__ __forceinline__ void page_pv(float (&o)[8][4], uint32_t vt, int valid
             const uint32_t sel = (i & 1) ? 0x7362u : 0x5140u;
             const uint32_t top = prmt(wa[i >> 1], wb[i >> 1], sel);   // tokens 2c, 2c+1
             const uint32_t bot = prmt(wc[i >> 1], wd[i >> 1], sel);   // tokens 2c+8, 2c+9
-            mma_16816(o[i], e4m3x2_to_half2(top), e4m3x2_to_half2(top >> 16),
-                      e4m3x2_to_half2(bot), e4m3x2_to_half2(bot >> 16), pb0, pb1);
+            uint32_t tl, th, bl, bh;
+            e4m3x4_to_half2x2(top, tl, th);
+            e4m3x4_to_half2x2(bot, bl, bh);
+            mma_16816(o[i], tl, th, bl, bh, pb0, pb1);
         }
     }
 }
@@ -204,7 +216,7 @@ __device__ __forceinline__ void softmax_step(WarpState& st, const float (&x)[kPa
 // (* k_scale for FP8).
 template <bool kFp8>
 __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t vt, int valid,
-                                            const uint32_t (&qf)[8][2], float sl, int lane) {
+                                            const QOperand<kFp8>& qf, float sl, int lane) {
     float x[1][4];
     page_logits<kFp8>(x[0], kt, valid, qf, sl, lane);
     uint32_t pb[2];
@@ -218,7 +230,7 @@ __device__ __forceinline__ void attend_page(WarpState& st, uint32_t kt, uint32_t
 // max, rescale and shuffles are paid once for 32 tokens.
 template <bool kFp8>
 __device__ __forceinline__ void attend_page_pair(WarpState& st, uint32_t ka, uint32_t va, uint32_t kb,
-                                                 uint32_t vb, int valid_b, const uint32_t (&qf)[8][2], float sl,
+                                                 uint32_t vb, int valid_b, const QOperand<kFp8>& qf, float sl,
                                                  int lane) {
     float x[2][4];
     page_logits<kFp8>(x[0], ka, kPageRows, qf, sl, lane);

@@ -19,6 +19,7 @@
 #include "fp8_scales.cuh"
 #include "qkv_proj.cuh"
 #include "prefill_attention.cuh"
+#include "prefill_tc.cuh"
 
 namespace {
 
@@ -47,6 +48,12 @@ constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 #endif
 #ifndef PKV_BAL_STAGES_FP8
 #define PKV_BAL_STAGES_FP8 4
+#endif
+// CTAs of one launch per SM (at most; fewer if they do not fit). One CTA per SM
+// leaves room, when its shared memory allows, for the next launch's CTA to
+// start its prologue beside it.
+#ifndef PKV_BAL_CTAS_PER_SM
+#define PKV_BAL_CTAS_PER_SM 8
 #endif
 constexpr int kBalWarpsF16 = PKV_BAL_WARPS_F16;
 constexpr int kBalWarpsFp8 = PKV_BAL_WARPS_FP8;
@@ -211,7 +218,7 @@ int balanced_grid(int B) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, BalShape<kFp8>::kThreads,
                                                       BalShape<kFp8>::smem_bytes(B)) != cudaSuccess)
         return 0;
-    return std::max(1, per_sm) * sms;
+    return std::max(1, std::min(per_sm, PKV_BAL_CTAS_PER_SM)) * sms;
 }
 
 struct BalancedLayout {
@@ -701,6 +708,38 @@ pkv_status launch_prefill(const pkv::PrefillParams& prm, const CUtensorMap& mk, 
                       prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// q [total, Hq, 128] f16 as a 3-D TMA tensor (channel, head, token) with
+// boxes of 64 channels x the G heads of one KV head x `tokens` tokens,
+// 128-byte swizzled: one box is the operand rows (token, head) of a prefill
+// tile for one half of the channels; tokens past `total` read as zeros.
+bool make_q_map(CUtensorMap* map, const void* q, int Hq, int total, int G, int tokens) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+    if (!encode) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hq, (cuuint64_t)total};
+    cuuint64_t strides[2] = {kHeadDim * 2, (cuuint64_t)Hq * kHeadDim * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)tokens};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// f16 prefill on tcgen05: one CTA per (tile of 128 / G query tokens, KV head,
+// sequence), one CTA per SM (its shared memory).
+pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
+                             int max_query_len, int Hkv, int B, cudaStream_t stream) {
+    using S = pkv::PrefillTcShape;
+    const int tokens = S::kRows / prm.G;
+    CUtensorMap mq;
+    if (!make_q_map(&mq, prm.q, prm.Hq, prm.total, prm.G, tokens)) return PKV_ERR_CUDA;
+    auto kernel = pkv::prefill_tc_kernel<0>;
+    static unsigned long long done = 0;
+    if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
+    const dim3 grid((unsigned)((max_query_len + tokens - 1) / tokens), (unsigned)Hkv, (unsigned)B);
+    return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm, tokens) == cudaSuccess
+               ? PKV_OK : PKV_ERR_CUDA;
+}
+
 bool ranges_overlap(const void* a, int64_t na, const void* b, int64_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return na > 0 && nb > 0 && x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
@@ -934,10 +973,12 @@ pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_c
     if (!cached_cache_map(&mk, k_cache, fp8, num_blocks, num_kv_heads) ||
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
         return PKV_ERR_CUDA;
-    const int chunks = (max_query_len + kPrefillConsumers - 1) / kPrefillConsumers;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return fp8 ? launch_prefill<true>(prm, mk, mv, chunks, num_kv_heads, batch, st)
-               : launch_prefill<false>(prm, mk, mv, chunks, num_kv_heads, batch, st);
+    if (!fp8) return launch_prefill_tc(prm, mk, mv, max_query_len, num_kv_heads, batch, st);
+    // an FP8 cache stays on the warp-level path: tcgen05 kind::f16 takes f16 operands only,
+    // and an E4M3 query would not meet the attention tolerance
+    const int chunks = (max_query_len + kPrefillConsumers - 1) / kPrefillConsumers;
+    return launch_prefill<true>(prm, mk, mv, chunks, num_kv_heads, batch, st);
 }
 
 pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_t num_q_heads,

@@ -121,6 +121,14 @@ __device__ __forceinline__ uint4 ld_stream_16(const uint4* src) {
     return v;
 }
 
+// 16-byte asynchronous copy global -> shared through L2 only (cp.async.cg),
+// its group commit, and the wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ---------------------------------------------------------- FP8 scales
 // Scale of KV head g from a device array of one element (per tensor) or one
 // per KV head.
@@ -212,6 +220,15 @@ __device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t two_codes) {
         "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
         : "=r"(d) : "r"(two_codes));
     return d;
+}
+
+// Four E4M3 codes (low byte first) to two f16x2: codes 0, 1 in `lo`, codes 2, 3
+// in `hi`. The 32-bit word is split into its 16-bit halves by register
+// aliasing, with no shift.
+__device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t four_codes, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi) : "r"(four_codes));
 }
 
 }  // namespace pkv

@@ -156,8 +156,8 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     const bool active = warp < nq;
     const int pos = L - n + qi;                  // its position
     const int64_t row = (int64_t)qs0 + qi;      // its row of q and out
-    uint32_t qf[8][2];
-    load_q_fragments<kFp8>(qf, active && r < G ? p.q + (row * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, c);
+    QOperand<kFp8> qf;
+    load_q_fragments(qf, active && r < G ? p.q + (row * p.Hq + (int64_t)g * G + r) * kHeadDim : nullptr, lane);
     WarpState st;
     st.reset();
 

@@ -102,3 +102,29 @@ def test_inconsistent_lengths_are_flagged_not_faulted():
     assert pkv.pkv_device_error() & pkv.DEVERR_CONTEXT_LEN
     assert (got[4:8] == 7.0).all()                  # the flagged sequence's rows are left alone
     assert np.isfinite(got[:4]).all() and np.isfinite(got[8:]).all()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (12, 4), (16, 4), (10, 2), (16, 2)])
+def test_prefill_group_sizes(Hq, Hkv):
+    """Every group size packs floor(128 / G) query tokens x G heads into the tile's rows
+    (128, 64, 42, 32, 25 and 16 tokens); several tiles per sequence, a one-query sequence."""
+    w, x, q, qs = _case("qwen2.5-1.5b", 9, [150, 1, 77], B=3, num_blocks=512, Hq=Hq, Hkv=Hkv,
+                        ctx=("uniform", 150, 600))
+    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), f"Hq {Hq} / Hkv {Hkv}")
+    assert pkv.pkv_device_error() == 0
+
+
+def test_prefill_large_logits():
+    """Logits that grow along the sequence: q scaled by 3 and each key by 1 + position / 256, so
+    the running maximum of a row rises by more than the rescale threshold (8 in the exp2 domain)
+    several times over its KV tiles and the output accumulated so far is rescaled each time."""
+    w, x, q, qs = _case("qwen2.5-7b", 10, [64, 200], B=2, num_blocks=1024, ctx=("uniform", 1500, 2000))
+    q = (q.astype(np.float32) * 3).astype(F16)
+    k = x["k_pool"].astype(np.float32)
+    for b, L in enumerate(x["context_lens"]):
+        for j in range(-(-int(L) // 16)):
+            pos = 16 * j + np.arange(16, dtype=np.float32)
+            k[x["block_tables"][b, j]] *= (1 + pos / 256)[:, None, None]
+    x["k_pool"] = k.astype(F16)                     # NaN rows stay NaN
+    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "large logits")
+    assert pkv.pkv_device_error() == 0
