@@ -31,23 +31,24 @@ constexpr int kStagesF16 = 3;   // 3 x 32 KiB ring: two CTAs per SM
 constexpr int kStagesFp8 = 6;   // 6 x 16 KiB ring
 
 // Balanced streaming kernel: worker warps per CTA and page slots per worker
-// ring (f16 pages are 8 KiB, FP8 pages 4 KiB), one CTA per SM (255 registers a
-// thread). Measured best on the benchmark workloads with two-page softmax
-// steps: f16 6 workers x 3 slots (144 KiB of ring; 8 x 3 took 17% longer on
-// the 1.5B-shaped step and 25% on the skewed one, 7B-shaped steps were within
-// 2% for 5..8 workers), FP8 8 workers x 4 slots (128 KiB; 8 x 6 and 7 x 6 were
-// slower). The macros exist for tuning builds.
+// ring (f16 pages are 8 KiB, FP8 pages 4 KiB), one CTA per SM. Measured best
+// on the benchmark workloads with two-page softmax steps: f16 6 workers x 3
+// slots (144 KiB of ring, 255 registers a thread; 8 x 3 took 17% longer on the
+// 1.5B-shaped step and 25% on the skewed one, 7B-shaped steps were within 2%
+// for 5..8 workers), FP8 12 workers x 3 slots (144 KiB; three warps per
+// scheduler at 168 registers, 2.5% faster than 8 x 4 at 255 registers, while
+// 10 x 4 and 10 x 3 were 10% slower). The macros exist for tuning builds.
 #ifndef PKV_BAL_WARPS_F16
 #define PKV_BAL_WARPS_F16 6
 #endif
 #ifndef PKV_BAL_WARPS_FP8
-#define PKV_BAL_WARPS_FP8 8
+#define PKV_BAL_WARPS_FP8 12
 #endif
 #ifndef PKV_BAL_STAGES_F16
 #define PKV_BAL_STAGES_F16 3
 #endif
 #ifndef PKV_BAL_STAGES_FP8
-#define PKV_BAL_STAGES_FP8 4
+#define PKV_BAL_STAGES_FP8 3
 #endif
 // CTAs of one launch per SM (at most; fewer if they do not fit). One CTA per SM
 // leaves room, when its shared memory allows, for the next launch's CTA to

@@ -23,21 +23,27 @@
 //  * One thread issues S = Q K^T (M = 128, N = 128, K = 128; K-major A and
 //    B) into TMEM columns [0, 128), and after the softmax O += P V (K = 128
 //    tokens; P K-major from shared memory, V MN-major) into columns
-//    [128, 256). S of tile j + 1 is issued before O += P V of tile j, so the
-//    tensor core works on one while the softmax warps work on the other.
+//    [128, 256) and l += P 1 (N = 16 against a tile of ones) into [256, 272),
+//    so the row sum is the sum of exactly the f16 probabilities the product
+//    used, accumulated in fp32 by the tensor core. S of tile j + 1 is issued
+//    before O += P V of tile j, so the tensor core works on one while the
+//    softmax warps work on the other.
 //  * Softmax: 8 warps, two per row quarter. Warp w serves rows (TMEM lanes)
 //    32 (w % 4) .. +31 and the half w / 4 of the columns: 64 tokens of S, 64
 //    channels of O, one 64-token chunk of P. Per tile a thread loads its
 //    half row of S, masks the causal edge (only on tiles that reach past the
 //    tile's first position), and takes the half row's maximum; the two halves
 //    of a row exchange maxima through shared memory (a barrier per pair of
-//    warps). The running maximum is raised only when a tile's maximum exceeds
-//    it by more than 8 (a factor 256 in the exp2 domain); then, and only then,
-//    the row of O is rescaled in TMEM. Probabilities are computed into
+//    warps). The running maximum (exp2 domain) is raised only when a tile's
+//    maximum exceeds it by more than 8 (a factor 256); then, and only then,
+//    the row of O and its l are rescaled in TMEM. A probability is
+//    exp2(s * scale - m): one fused multiply-add and the fp32 exp2, rounded to
+//    f16. (The two-wide f16 exp2 would halve the multi-function unit's work,
+//    but its f16 argument, 2^-9 apart near -8, moved outputs of magnitude
+//    about 4 past the 2e-3 bound.) Probabilities are computed into
 //    registers first; once O += P V of the previous tile has completed (its
 //    P buffer is then free, and O may be rescaled) they are written to shared
-//    memory as f16 in the operand layout. The row sum l adds the same f16
-//    values, and the final O / l is written to out as f16.
+//    memory as f16 in the operand layout. The output is O / l in f16.
 //  * Rows past the context in the sequence's last page (free slots, any
 //    content) are zeroed in shared memory before their V is used; pages past
 //    the tile's last position are loaded from outside the pool, which TMA
@@ -53,29 +59,6 @@
 
 namespace pkv {
 
-// One in PKV_PREFILL_POLY_EVERY probability pairs is exponentiated on the FMA
-// pipe (exp2_poly3) instead of the multi-function unit, whose throughput (16
-// results per clock per SM) otherwise equals the tensor core's time per tile.
-// 0: all on the multi-function unit. A tuning switch.
-#ifndef PKV_PREFILL_POLY_EVERY
-#define PKV_PREFILL_POLY_EVERY 0
-#endif
-
-// 2^x for x <= 8 on the FMA pipe: Cody-Waite reduction x = n + f with n the
-// nearest integer (by the 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5],
-// 2^f by a degree-3 polynomial fitted here for least maximum relative error on
-// that interval (7.5e-5 including fp32 evaluation, below the 2^-11 of the f16
-// rounding that follows), and 2^n added to the exponent field. Arguments below
-// -126 (masked entries are -inf) give about 2^-126, which rounds to 0 in f16.
-__device__ __forceinline__ float exp2_poly3(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.05517150089144707f, f, 0.24261096119880676f), f, 0.6932609677314758f), f,
-                         0.9999280571937561f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 struct PrefillTcShape {
     static constexpr int kRows = 128;                  // M: query tokens x heads
     static constexpr int kKvTok = 128;                 // N of S, K of P V: tokens per KV tile
@@ -86,11 +69,12 @@ struct PrefillTcShape {
     static constexpr int kPBytes = 2 * kChunk;         // P: 128 rows x 128 tokens (one buffer)
     static constexpr int kBarBytes = 256;
     static constexpr int kXchgBytes = 2 * 2 * 128 * 4;  // per-half row values, two buffers
-    static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kKvBytes + kPBytes + kBarBytes + kXchgBytes;
+    static constexpr int kOnesBytes = 2 * 16 * 128;    // 16 rows x 128 tokens of f16 ones (K-major, N = 16)
+    static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kKvBytes + kPBytes + kOnesBytes + kBarBytes + kXchgBytes;
     static constexpr int kSoftmaxWarps = 8;
     static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);   // warps 0-7 softmax, 8 TMA K (and Q), 9 TMA V, 10 MMA
     static constexpr int kTmaKWarp = kSoftmaxWarps, kTmaVWarp = kSoftmaxWarps + 1, kMmaWarp = kSoftmaxWarps + 2;
-    static constexpr uint32_t kTmemCols = 256;         // S [0, 128), O [128, 256)
+    static constexpr uint32_t kTmemCols = 512;         // S [0, 128), O [128, 256), l [256, 272)
     static constexpr float kRescaleThreshold = 8.f;    // log2 of the largest unnormalised probability
 };
 
@@ -132,7 +116,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto k_s = [&](int s) { return base + S::kQBytes + s * S::kKvBytes; };
     auto v_s = [&](int s) { return k_s(s) + 2 * S::kChunk; };
     const uint32_t p_s = base + S::kQBytes + S::kStages * S::kKvBytes;
-    const uint32_t bars = p_s + S::kPBytes;
+    const uint32_t ones_s = p_s + S::kPBytes;                        // [2 token halves][16 rows][128 B]
+    const uint32_t bars = ones_s + S::kOnesBytes;
     const uint32_t q_full = bars, s_full = bars + 8, s_free = bars + 16, o_done = bars + 24, drain = bars + 32;
     // K and V stages: full (TMA landed) and empty (the MMA that read it is done)
     auto k_full = [&](int s) { return bars + 40 + 8u * s; };
@@ -140,10 +125,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto v_full = [&](int s) { return bars + 184 + 8u * s; };
     auto v_empty = [&](int s) { return bars + 200 + 8u * s; };
     const uint32_t p_full = bars + 72;
-    // pair barriers: the two warps of row quarter q meet at xchg(q, j & 1) every
-    // tile and at xchg_fin(q) at the end
+    // pair barriers: the two warps of row quarter q meet at xchg(q, j & 1) every tile
     auto xchg = [&](int q, int i) { return bars + 88 + 8u * (2 * q + i); };
-    auto xchg_fin = [&](int q) { return bars + 152 + 8u * q; };
     const uint32_t tmem_slot = bars + 248;
     float* red = reinterpret_cast<float*>(smem_raw + (bars + S::kBarBytes - raw));   // [2][2 halves][128 rows]
 
@@ -165,7 +148,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int q = 0; q < 4; ++q) {
             mbar_init(xchg(q, 0), 64);
             mbar_init(xchg(q, 1), 64);
-            mbar_init(xchg_fin(q), 64);
         }
         mbar_init_fence();
     }
@@ -174,6 +156,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t a = q_s + (part >> 3) * S::kChunk + r * 128 + (part & 7) * 16;
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(a), "r"(0u) : "memory");
     }
+    for (int i = threadIdx.x; i < S::kOnesBytes / 16; i += S::kThreads)     // f16 1.0 pairs
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(ones_s + 16 * i), "r"(0x3C003C00u) : "memory");
     fence_proxy_async_shared();
     if (warp == S::kMmaWarp) {
         tmem_alloc(tmem_slot, S::kTmemCols);
@@ -184,7 +168,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     uint32_t tmem;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_slot) : "memory");
-    const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
+    const uint32_t tmem_s = tmem, tmem_o = tmem + 128, tmem_l = tmem + 256;
 
     // Bounded wait that also gives up once another role has given up.
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -249,6 +233,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ================================ MMA ================================
         constexpr uint32_t kIdescS = umma_idesc_f16(128, 128, 0);    // Q K^T: both K-major
         constexpr uint32_t kIdescPV = umma_idesc_f16(128, 128, 1);   // P V: V is MN-major
+        constexpr uint32_t kIdescL = umma_idesc_f16(128, 16, 0);     // P 1: the row sums
         const int last_page = (L - 1) / kPageRows;
         const int valid_last = L - last_page * kPageRows;            // live rows of that page
         auto issue_pv = [&](int jp) -> bool {
@@ -275,6 +260,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint64_t a = umma_desc_sw128(p_s + (kk >> 2) * S::kChunk + (kk & 3) * 32, 16, 1024);
                     const uint64_t bdesc = umma_desc_sw128(v_s(s) + kk * 2048, S::kChunk, 1024);
                     umma_f16_ss(tmem_o, a, bdesc, kIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = umma_desc_sw128(p_s + (kk >> 2) * S::kChunk + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bdesc = umma_desc_sw128(ones_s + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+                    umma_f16_ss(tmem_l, a, bdesc, kIdescL, (jp > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(o_done);
                 umma_commit(v_empty(s));
@@ -316,7 +307,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const uint32_t s_cols = tmem_s + lane_base + 64 * half, o_cols = tmem_o + lane_base + 64 * half;
         const float sl = p.logit_scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY;                            // running maximum, exp2 domain (s * sl)
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
             if (!(ok = __all_sync(0xffffffffu, wait(s_full, j & 1)))) break;
@@ -326,23 +317,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tmem_ld32(s_cols + 32, *reinterpret_cast<float(*)[32]>(x + 32));
             tc_fence_before();
             mbar_arrive(s_free);
-            // scale, causal mask, maximum of the half row (four independent chains)
+            // causal mask and maximum of the half row's raw logits (four independent chains);
+            // the scale sl > 0 is applied to the maximum and inside the exponent's multiply-add
             const int t0 = j * S::kKvTok + 64 * half;
+            const bool edge = j * S::kKvTok + S::kKvTok - 1 > pos0;   // some entries past a row's position
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (j * S::kKvTok + S::kKvTok - 1 > pos0) {
+            if (edge) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    x[c] = t0 + c <= prow ? x[c] * sl : -INFINITY;
-                    mx[c & 3] = fmaxf(mx[c & 3], x[c]);
-                }
+                for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], t0 + c <= prow ? x[c] : -INFINITY);
             } else {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    x[c] *= sl;
-                    mx[c & 3] = fmaxf(mx[c & 3], x[c]);
-                }
+                for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], x[c]);
             }
             float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            mt = mt > -INFINITY ? mt * sl : -INFINITY;       // (a zero scale must not make -inf * 0)
             // the row's maximum: exchange with the other half of the row
             red[(j & 1) * 256 + half * 128 + r] = mt;
             mbar_arrive(xchg(quarter, j & 1));
@@ -351,22 +339,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // running maximum, raised only by more than the threshold
             const bool raise = mt > m_run + S::kRescaleThreshold;
             const float m_new = raise ? mt : m_run;
-            // probabilities of this half row, f16 pairs (tokens 64 half + 2i, + 1)
+            // probabilities of this half row as f16 pairs (tokens 64 half + 2i, + 1):
+            // exp2(s * sl - m_new), one fused multiply-add and the fp32 exp2; masked entries give 0
             uint32_t w[32];
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                if (PKV_PREFILL_POLY_EVERY > 0 && i % (PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1) ==
-                                                      (PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1) - 1)
-                    w[i] = pack_half2(exp2_poly3(x[2 * i] - m_new), exp2_poly3(x[2 * i + 1] - m_new));
-                else
-                    w[i] = pack_half2(fast_exp2(x[2 * i] - m_new), fast_exp2(x[2 * i + 1] - m_new));
-                // l sums the f16 probabilities the P V product uses, so that a dominant
-                // probability's rounding cancels in O / l
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-                rs[i & 3] += f.x + f.y;
+                float e0 = fmaf(x[2 * i], sl, -m_new), e1 = fmaf(x[2 * i + 1], sl, -m_new);
+                if (edge) {
+                    e0 = t0 + 2 * i <= prow ? e0 : -INFINITY;
+                    e1 = t0 + 2 * i + 1 <= prow ? e1 : -INFINITY;
+                }
+                w[i] = pack_half2(fast_exp2(e0), fast_exp2(e1));
             }
-            // O += P V of the previous tile has completed: the P buffer is free and O final for it
+            // O += P V of the previous tile has completed: the P buffer is free and O, l final for it
             if (j > 0) {
                 if (!(ok = __all_sync(0xffffffffu, wait(o_done, (j - 1) & 1)))) break;
                 tc_fence_after();
@@ -382,12 +367,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int i = 0; i < 32; ++i) o[i] *= alpha;
                     tmem_st32(o_cols + 32 * c, o);
                 }
+                if (half == 0) tmem_st1(tmem_l + lane_base, tmem_ld1(tmem_l + lane_base) * alpha);
                 tmem_wait_st();
-                l_run *= alpha;
                 corrected = true;
             }
             m_run = m_new;
-            l_run += (rs[0] + rs[1]) + (rs[2] + rs[3]);
             // chunk `half` of row r of P: K-major operand layout, 16-byte pieces of 8 tokens
             const uint32_t prow_addr = p_s + half * S::kChunk + r * 128;
 #pragma unroll
@@ -400,18 +384,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (corrected) tc_fence_before();
             mbar_arrive(p_full);
         }
-        // ---- out = O / l, l summed over both halves of the row ----
-        // (the buffer of tile ntiles - 2, which both warps of the pair have read)
-        float* lx = red + (ntiles & 1) * 256;
-        if (ok) {
-            lx[half * 128 + r] = l_run;
-            mbar_arrive(xchg_fin(quarter));
-            ok = __all_sync(0xffffffffu, wait(xchg_fin(quarter), 0));
-        }
+        // ---- out = O / l ----
         if (ok) ok = __all_sync(0xffffffffu, wait(o_done, (ntiles - 1) & 1));
         if (ok) {
             tc_fence_after();
-            const float inv = p.out_scale / (l_run + lx[(half ^ 1) * 128 + r]);
+            const float inv = p.out_scale / tmem_ld1(tmem_l + lane_base);
             __half* dst = p.out + ((int64_t)(qs0 + i0 + ti) * p.Hq + (int64_t)g * G + hh) * kHeadDim + 64 * half;
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {

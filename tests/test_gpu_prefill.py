@@ -128,3 +128,12 @@ def test_prefill_large_logits():
     x["k_pool"] = k.astype(F16)                     # NaN rows stay NaN
     assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "large logits")
     assert pkv.pkv_device_error() == 0
+
+
+def test_prefill_zero_scale_is_the_causal_mean():
+    """softmax_scale = 0: every query averages V over its causal window (masked entries stay out
+    of the average even though 0 times their logit is 0)."""
+    w, x, q, qs = _case("qwen2.5-7b", 11, [40, 150], B=2, num_blocks=512, ctx=("uniform", 200, 400))
+    x["softmax_scale"] = np.float32(0.0)
+    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "zero scale")
+    assert pkv.pkv_device_error() == 0
