@@ -251,7 +251,8 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
 
 /*
  * fused_add_rmsnorm_qkv -- the step before attention, fused: residual add,
- * RMSNorm and the QKV projection of num_tokens decode tokens in one launch,
+ * RMSNorm and the QKV projection of num_tokens decode tokens in one launch
+ * (tcgen05 tensor cores, split-K over a thread-block cluster),
  * writing q in the layout paged_gqa_decode_attention / _step take and k_new,
  * v_new in the layout the cache write and the fused step take.
  *
@@ -278,11 +279,11 @@ pkv_status paged_gqa_decode_step(void* out, const void* q, const void* k_new, co
  * update `residual` in place: other CTAs still read it).
  *
  * Precision: residual_out is exact (bit-for-bit the rounded sum). q, k_new,
- * v_new are f16 (nearest even) of an fp32-accumulated dot product whose
- * activation operand is f16(s * gamma * 2^-e_t), e_t a per-token power of
- * two chosen so that no operand overflows; the 1/RMS factor is applied in
- * fp32 after the sum. The error is within 2^-10 * sum_k |w[n][k] y[t][k]|
- * plus the output rounding.
+ * v_new are f16 (nearest even) of an fp32-accumulated dot product of s (exact
+ * in f16) with the weight row scaled by gamma and rounded once to f16,
+ * f16(w[n][k] * gamma[k]); the 1/RMS factor is applied in fp32 after the sum.
+ * The error is within 2^-10 * sum_k |w[n][k] y[t][k]| plus the output
+ * rounding, provided no |w[n][k] * gamma[k]| exceeds 65504.
  *
  * Supported: H a multiple of 64 and at most 8192, D a multiple of 8,
  * N <= 2^24, T <= 4194240; others return PKV_ERR_UNSUPPORTED. eps must be
@@ -340,9 +341,10 @@ pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_c
 /*
  * fused_add_rmsnorm_qkv_plan -- the launch plan fused_add_rmsnorm_qkv uses on
  * the current device for these sizes, for reports and tuning. Writes five
- * int32 to plan (host memory): weight-tile rows, slices of the hidden size per
- * cluster, feature tiles per CTA, CTAs, token tiles of 64. Host-only (queries
- * the device's cluster occupancy); PKV_ERR_UNSUPPORTED as the projection.
+ * int32 to plan (host memory): weight-tile rows (128), slices of the hidden
+ * size per cluster (split-K), tokens per token tile (64, 128 or 256), CTAs,
+ * token tiles. Host-only (queries the device's cluster occupancy);
+ * PKV_ERR_UNSUPPORTED as the projection.
  */
 pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_t num_q_heads,
                                       int32_t num_kv_heads, int32_t head_dim, int32_t* plan);

@@ -375,7 +375,7 @@ def fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D) -> dict:
     """The launch plan of fused_add_rmsnorm_qkv for these sizes on the current device."""
     plan = (ctypes.c_int32 * 5)()
     _check(load_library().fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D, plan), "fused_add_rmsnorm_qkv_plan")
-    return dict(zip(("tile_rows", "slices", "tiles_per_cta", "ctas", "token_tiles"), list(plan)))
+    return dict(zip(("tile_rows", "slices", "token_tile", "ctas", "token_tiles"), list(plan)))
 
 
 def paged_gqa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start, *,

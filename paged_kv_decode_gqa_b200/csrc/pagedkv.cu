@@ -547,42 +547,36 @@ pkv_status check_device_scales(const float* k_scales, const float* v_scales, int
 }
 
 // ------------------------------------------------ fused add + RMSNorm + QKV
-// One CTA shape per weight-tile height: 128 rows with a 4-slot ring (16 KiB
-// slots), 256 rows with a 3-slot ring (32 KiB slots); the rest of the shared
-// memory holds the activation slice.
-constexpr int kQkvStages1 = 4;
-constexpr int kQkvStages2 = 3;
 constexpr int kQkvMaxSplit = pkv::kQkvMaxCluster;   // portable cluster size
-template <int kMT>
-using QkvShapeT = pkv::QkvShape<kMT, kMT == 1 ? kQkvStages1 : kQkvStages2>;
-template <int kMT>
-auto qkv_kernel() { return pkv::add_rmsnorm_qkv_kernel<kMT, kMT == 1 ? kQkvStages1 : kQkvStages2>; }
+constexpr int kQkvMaxHidden = 8192;
 
-// W [N, H] f16 as a 2-D TMA tensor (k, feature) with [rows x 64] boxes,
-// 128-byte swizzled; rows past N read as zeros.
-bool make_w_map(CUtensorMap* map, const void* w, int H, int N, int rows) {
+// A [rows, H] f16 matrix as a 2-D TMA tensor (k, row) with [box_rows x 64]
+// boxes, 128-byte swizzled (the UMMA K-major layout); rows past the end read
+// as zeros.
+bool make_rows_map(CUtensorMap* map, const void* ptr, int H, int rows, int box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
     if (!encode) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)H, (cuuint64_t)N};
+    cuuint64_t dims[2] = {(cuuint64_t)H, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)H * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)rows};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct QkvPlan {
-    int mt = 0, split = 0, slab_blocks = 0, ftiles = 0, tiles_per_cta = 0, runs = 0, ttiles = 0;
+    int acc = 0, split = 0, tt = 0, stages = 0, mtiles = 0, ttiles = 0;
     size_t smem = 0;
     double cost = 0;
 };
 
-template <int kMT>
+auto qkv_kernel(int acc) { return acc == 1 ? pkv::rmsnorm_qkv_kernel<1> : pkv::rmsnorm_qkv_kernel<2>; }
+
 cudaLaunchConfig_t qkv_config(const QkvPlan& pl, cudaStream_t st, cudaLaunchAttribute (&attr)[2]) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(pl.runs * pl.split), (unsigned)pl.ttiles);
-    cfg.blockDim = dim3(QkvShapeT<kMT>::kThreads);
+    cfg.gridDim = dim3((unsigned)(pl.mtiles * pl.split), (unsigned)pl.ttiles);
+    cfg.blockDim = dim3(pkv::QkvShape::kThreads);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -596,67 +590,14 @@ cudaLaunchConfig_t qkv_config(const QkvPlan& pl, cudaStream_t st, cudaLaunchAttr
     return cfg;
 }
 
-// The best plan for one tile height. For each split of H (from the fewest
-// slices whose activations fit in shared memory up to the cluster limit) that
-// the device can schedule as a cluster, and each run length (feature tiles per
-// CTA), a cost in W-byte equivalents per CTA times the waves:
-//   run * tile rows * slice * 2      W streamed
-// + 7 * 64 * slice                   building the activation slice (measured:
-//                                    about 0.3 SM cycles an element, where W
-//                                    streams at about 25 bytes an SM cycle)
-// + run * 40000                      a tile's cluster reduction
-// Returns false if no split fits.
-template <int kMT>
-bool qkv_candidate(int T, int H, int N, int sms, QkvPlan* out) {
-    using S = QkvShapeT<kMT>;
-    static unsigned long long done = 0;
-    auto kernel = qkv_kernel<kMT>();
-    if (ensure_smem(kernel, (int)S::smem_bytes(S::kMaxSlabBlocks), &done) != cudaSuccess) return false;
-    const int kb = H / 64;
-    const int ftiles = (N + S::kFT - 1) / S::kFT;
-    const int ttiles = (T + S::kTT - 1) / S::kTT;
-    const int split_min = (kb + S::kMaxSlabBlocks - 1) / S::kMaxSlabBlocks;
-    const int split_max = std::min(kQkvMaxSplit, kb);
-    bool found = false;
-    for (int split = split_min; split <= split_max; ++split) {
-        QkvPlan pl;
-        pl.mt = kMT;
-        pl.split = split;
-        pl.slab_blocks = (kb + split - 1) / split;
-        pl.smem = S::smem_bytes(pl.slab_blocks);
-        pl.ftiles = ftiles;
-        pl.ttiles = ttiles;
-        pl.tiles_per_cta = 1;
-        pl.runs = ftiles;
-        cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = qkv_config<kMT>(pl, nullptr, attr);
-        int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) {
-            (void)cudaGetLastError();
-            continue;
-        }
-        if (clusters < 1) continue;
-        const int64_t slots = std::max<int64_t>(1, std::min<int64_t>((int64_t)clusters * split, sms));
-        for (int runs = ftiles; runs >= 1; --runs) {
-            const int per = (ftiles + runs - 1) / runs;
-            if ((ftiles + per - 1) / per != runs) continue;       // only the tightest run length per count
-            const int64_t ctas = (int64_t)runs * ttiles * split;
-            const int64_t waves = (ctas + slots - 1) / slots;
-            const double slice = 64.0 * pl.slab_blocks;
-            const double cost = (double)waves * (per * (double)S::kFT * slice * 2 + 7.0 * 64 * slice + per * 40000.0);
-            if (!found || cost < out->cost) {
-                pl.tiles_per_cta = per;
-                pl.runs = runs;
-                pl.cost = cost;
-                *out = pl;
-                found = true;
-            }
-        }
-    }
-    return found;
-}
-
+// The plan: token tiles of 64, 128 or 256 tokens (the MMA's N), feature
+// tiles of 128 or 256 rows, and the split of H (cluster size). An SM keeps
+// its ring's bytes in flight, so a CTA's time goes with the bytes it streams:
+// cost = waves x (stages streamed x stage bytes + a share per cluster rank
+// for the reduction), waves counted from the clusters the device reports it
+// can hold at once.
 bool qkv_plan(int T, int H, int N, QkvPlan* out) {
+    using S = pkv::QkvShape;
     struct Entry {
         int dev, T, H, N;
         QkvPlan plan;
@@ -664,33 +605,81 @@ bool qkv_plan(int T, int H, int N, QkvPlan* out) {
     constexpr int kSlots = 8;
     thread_local Entry cache[kSlots];
     thread_local int used = 0, next = 0;
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
     for (int i = 0; i < used; ++i)
         if (cache[i].dev == dev && cache[i].T == T && cache[i].H == H && cache[i].N == N) {
             *out = cache[i].plan;
             return true;
         }
-    QkvPlan a, b;
-    const bool ha = qkv_candidate<1>(T, H, N, sms, &a);
-    const bool hb = qkv_candidate<2>(T, H, N, sms, &b);
-    if (!ha && !hb) return false;
-    *out = (ha && (!hb || a.cost <= b.cost)) ? a : b;
+    static unsigned long long done1 = 0, done2 = 0;
+    if (ensure_smem(qkv_kernel(1), S::kSmemMax, &done1) != cudaSuccess ||
+        ensure_smem(qkv_kernel(2), S::kSmemMax, &done2) != cudaSuccess)
+        return false;
+    const int kb = H / 64;
+    const int tt = T <= 64 ? 64 : T <= 128 ? 128 : 256;
+    const int ttiles = (T + tt - 1) / tt;
+    bool found = false;
+    for (int acc = 1; acc <= 2; ++acc) {
+        const int m = 128 * acc;
+        for (int split = 1; split <= std::min(kQkvMaxSplit, kb); ++split) {
+            QkvPlan pl;
+            pl.acc = acc;
+            pl.split = split;
+            pl.tt = tt;
+            pl.mtiles = (N + m - 1) / m;
+            pl.ttiles = ttiles;
+            const size_t fixed = 1024 + S::kHeader + (size_t)S::gamma_bytes(kb, split);
+            const int stage = S::stage_bytes(m, tt);
+            pl.stages = (int)std::min<size_t>(pkv::kQkvMaxStages, (S::kSmemMax - fixed) / stage);
+            // at least two stages, and the partial tile [tt][m] fp32 fits in the ring it reuses
+            if (pl.stages < 2 || (size_t)pl.stages * stage < (size_t)tt * m * 4) continue;
+            pl.smem = S::smem_bytes(m, tt, pl.stages, kb, split);
+            cudaLaunchAttribute attr[2];
+            cudaLaunchConfig_t cfg = qkv_config(pl, nullptr, attr);
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, qkv_kernel(acc), &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                continue;
+            }
+            if (clusters < 1) continue;
+            const int64_t waves = ((int64_t)pl.mtiles * ttiles + clusters - 1) / clusters;
+            const int per = (kb + split - 1) / split;
+            pl.cost = (double)waves * ((double)per * stage + 16384.0 * split);
+            if (!found || pl.cost < out->cost) {
+                *out = pl;
+                found = true;
+            }
+        }
+    }
+    if (!found) return false;
     cache[next] = Entry{dev, T, H, N, *out};
     next = (next + 1) % kSlots;
     used = std::min(used + 1, kSlots);
     return true;
 }
 
-template <int kMT>
-pkv_status launch_qkv(const QkvPlan& pl, const pkv::QkvParams& prm, const void* w, cudaStream_t st) {
-    CUtensorMap map;
-    if (!make_w_map(&map, w, prm.H, prm.N, QkvShapeT<kMT>::kFT)) return PKV_ERR_CUDA;
+// Two launches: s = x + r into residual_out, then the projection, which reads
+// s back (from L2) and may request its first W tiles while the add runs.
+pkv_status launch_qkv(const QkvPlan& pl, const pkv::QkvParams& prm, const void* w, const void* x,
+                      const void* residual, cudaStream_t st) {
+    CUtensorMap mw, ms;
+    if (!make_rows_map(&mw, w, prm.H, prm.N, 128 * pl.acc) ||
+        !make_rows_map(&ms, prm.residual_out, prm.H, prm.T, pl.tt))
+        return PKV_ERR_CUDA;
+    const int64_t chunks = (int64_t)prm.T * prm.H / 8;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const int64_t blocks = std::min<int64_t>((chunks + 255) / 256, (int64_t)sms * 4);
+    if (launch_pdl(pkv::add_residual_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                   static_cast<const __half*>(x), static_cast<const __half*>(residual), prm.residual_out,
+                   chunks) != cudaSuccess)
+        return PKV_ERR_CUDA;
     cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = qkv_config<kMT>(pl, st, attr);
-    return cudaLaunchKernelEx(&cfg, qkv_kernel<kMT>(), map, prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    cudaLaunchConfig_t cfg = qkv_config(pl, st, attr);
+    return cudaLaunchKernelEx(&cfg, qkv_kernel(pl.acc), mw, ms, prm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ paged prefill
@@ -987,15 +976,15 @@ pkv_status fused_add_rmsnorm_qkv_plan(int32_t num_tokens, int32_t hidden, int32_
     if (!plan || num_tokens <= 0 || hidden <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return PKV_ERR_INVALID_ARG;
     const int64_t N = ((int64_t)num_q_heads + 2 * (int64_t)num_kv_heads) * head_dim;
-    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxSplit * 64 * QkvShapeT<1>::kMaxSlabBlocks ||
-        N > (1 << 24) || num_tokens > 65535 * 64)
+    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxHidden || N > (1 << 24) ||
+        num_tokens > 65535 * 64)
         return PKV_ERR_UNSUPPORTED;
     QkvPlan pl;
     if (!qkv_plan(num_tokens, hidden, (int)N, &pl)) return PKV_ERR_CUDA;
-    plan[0] = 128 * pl.mt;
+    plan[0] = 128 * pl.acc;
     plan[1] = pl.split;
-    plan[2] = pl.tiles_per_cta;
-    plan[3] = pl.runs * pl.split * pl.ttiles;
+    plan[2] = pl.tt;
+    plan[3] = pl.mtiles * pl.split * pl.ttiles;
     plan[4] = pl.ttiles;
     return PKV_OK;
 }
@@ -1017,8 +1006,8 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
         if ((num_tokens > 0 && !ptr) || !aligned16(ptr)) return PKV_ERR_INVALID_ARG;
     if (bias && !aligned16(bias)) return PKV_ERR_INVALID_ARG;
     const int64_t N = ((int64_t)num_q_heads + 2 * (int64_t)num_kv_heads) * head_dim;
-    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxSplit * 64 * QkvShapeT<1>::kMaxSlabBlocks ||
-        N > (1 << 24) || num_tokens > 65535 * 64)
+    if (head_dim % 8 != 0 || hidden % 64 != 0 || hidden > kQkvMaxHidden || N > (1 << 24) ||
+        num_tokens > 65535 * 64)
         return PKV_ERR_UNSUPPORTED;
     const int64_t T = num_tokens;
     const int64_t act = T * hidden * 2, qb = T * num_q_heads * head_dim * 2, kvb = T * num_kv_heads * head_dim * 2;
@@ -1034,8 +1023,6 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
     QkvPlan pl;
     if (!qkv_plan(num_tokens, hidden, (int)N, &pl)) return PKV_ERR_CUDA;
     pkv::QkvParams prm;
-    prm.x = static_cast<const __half*>(x);
-    prm.residual = static_cast<const __half*>(residual);
     prm.gamma = static_cast<const __half*>(gamma);
     prm.bias = static_cast<const __half*>(bias);
     prm.residual_out = static_cast<__half*>(residual_out);
@@ -1049,13 +1036,11 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
     prm.kv_cols = num_kv_heads * head_dim;
     prm.kblocks = hidden / 64;
     prm.split = pl.split;
-    prm.slab_blocks = pl.slab_blocks;
-    prm.ftiles = pl.ftiles;
-    prm.tiles_per_cta = pl.tiles_per_cta;
+    prm.tt = pl.tt;
+    prm.stages = pl.stages;
     prm.eps = eps;
     prm.prefetch_w = (flags & PKV_STEP_OVERLAP_PREVIOUS) ? 1 : 0;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return pl.mt == 1 ? launch_qkv<1>(pl, prm, w_qkv, st) : launch_qkv<2>(pl, prm, w_qkv, st);
+    return launch_qkv(pl, prm, w_qkv, x, residual, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

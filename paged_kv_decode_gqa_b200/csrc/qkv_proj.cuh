@@ -1,51 +1,66 @@
-// Fused residual add + RMSNorm + QKV projection of one decode step.
+// Fused residual add + RMSNorm + QKV projection of one decode step, on the
+// fifth-generation tensor cores (tcgen05, TMEM accumulators).
 //
 // "rvLLM 소개" (discuss.pytorch.kr), §퓨즈드 CUDA 커널: each layer runs the
-// residual add, the RMSNorm and the QKV projection as one kernel, so the
-// normalised activations never travel through HBM. For T decode tokens:
+// residual add, the RMSNorm and the QKV projection fused, so the normalised
+// activations never travel through HBM. For T decode tokens:
 //   s   = f16(x + residual)                 returned: the new residual stream
 //   y   = s / sqrt(mean(s^2) + eps) * gamma
 //   qkv = W y + bias                        W [N, H] f16, rows q heads | k | v
 // and q, k, v leave in the layouts the cache write and the decode step take.
 //
 // At decode batch sizes this is a thin GEMM (N = 2048..4608 features, T =
-// 64..256 tokens, K = H = 1536..3584) whose bytes are almost all W, so the
-// grid reads W once from HBM and keeps the activations on chip:
-//  * A CTA owns 64 tokens x one slice of H and streams W for a run of
-//    consecutive feature tiles of kFT = 128 * kMT rows against them, so the
-//    activation slice is built once for several tiles. The `split` slices of
-//    a run are one thread-block cluster (split-K); after each feature tile
-//    their partial sums meet in distributed shared memory, in rank order.
-//  * W tiles [kFT rows x 64 k] come by TMA (128-byte swizzle) into a ring of
-//    kStages slots that runs on across the feature tiles. With the overlap
-//    flag the first ones are requested before the grid-dependency wait (W is
-//    not written by the previous launch).
-//  * The slice's activations are built once in shared memory: s = x + r in
-//    f16 (stored to residual_out by the CTAs of the first run), the token's
-//    sum of squares in fp32 and max |s| in f16, then the tensor-core operand
-//    b = f16(s * gamma * 2^-e_t) with e_t the per-token power of two that puts
-//    max |s| * max |gamma| (over the slice) in [2^14, 2^15). The division by
-//    the RMS happens after the sum (the RMS needs all slices), so the operand
-//    is scaled to neither overflow nor lose precision: s * gamma alone passes
-//    65504 in residual streams with large channels.
-//  * mma.sync m16n8k16 with features on M and tokens on N, fp32 accumulators.
-//  * After each feature tile: partial * 2^e_t into shared memory; cluster
-//    barrier; rank r sums its share of the tile's tokens over all ranks,
-//    multiplies by 1 / sqrt(sum_s^2 / H + eps) (IEEE sqrt and division), adds
-//    the bias and stores f16 (round to nearest even); cluster barrier.
+// 64..256 tokens, K = H = 1536..3584) whose bytes are almost all W. Each SM
+// keeps a fixed number of bytes in flight (its shared-memory ring), so the
+// time is set by the bytes each SM must bring in; the design minimises them:
+//  * Two launches. `add_residual_kernel` forms s = x + r (one f16 rounding,
+//    nearest even) into residual_out, which the caller receives anyway. The
+//    projection then reads one activation tile per k block (s, from L2)
+//    instead of two (x and r), and every 128- or 256-feature tile reads it.
+//    The projection is launched with programmatic dependent launch and, with
+//    the overlap flag, requests its first W tiles while the add still runs.
+//  * The normalisation is folded into the operands and the epilogue, never
+//    materialised: 1/RMS is a per-token scalar applied after the sum, and
+//    gamma scales the weight tile instead of the activations:
+//      qkv[t][n] = (1 / rms_t) * sum_k f16(W[n][k] * gamma[k]) * s[t][k].
+//    The activation operand is s itself, exact in f16 (no per-token scale,
+//    no overflow); W * gamma is rounded once to f16 (relative 2^-11, as
+//    rounding the activations would be).
+//  * Work unit: (M = 128 or 256 features, token tile of TT = 64, 128 or 256
+//    tokens, slice of H). The `split` slices of one (features, tokens) tile
+//    are one thread-block cluster (split-K); their fp32 partial tiles meet in
+//    distributed shared memory at the end.
+//  * Per k block, one TMA warp brings the W tile [M rows x 64 k] and the s
+//    tile [TT tokens x 64 k] (128-byte swizzle, the UMMA K-major layout) into
+//    one stage of a ring. Eight warps multiply the W tile by gamma in place
+//    and add each token's s^2 to its sum in fp32. One thread issues, per
+//    128-row half of the W tile, D[128 x TT] += W' s^T (4 steps of K = 16,
+//    `tcgen05.mma.kind::f16`) into its own TMEM columns and commits the
+//    stage back to the TMA warp.
+//  * Epilogue: the eight warps read the accumulators out of TMEM into shared
+//    memory as fp32 [token][feature]; after a cluster barrier, rank r sums
+//    its share of the tile's tokens over all ranks in rank order (every
+//    remote load of two items in flight before the first sum), and the sums
+//    of squares likewise, multiplies by 1 / sqrt(sum_s^2 / H + eps) (IEEE
+//    square root and division), adds the bias and stores f16 (nearest even);
+//    a second cluster barrier keeps every partial tile alive until its
+//    readers are done.
+// Every barrier wait has a time limit; one that runs out flags
+// PKV_DEVERR_WAIT_TIMEOUT, and every role stops, waits for what it has in
+// flight, still takes both cluster barriers, and TMEM is freed.
 #pragma once
 
 #include <cooperative_groups.h>
 
 #include "pkv_device.cuh"
+#include "umma.cuh"
 
 namespace pkv {
 
 constexpr int kQkvMaxCluster = 8;
+constexpr int kQkvMaxStages = 8;
 
 struct QkvParams {
-    const __half* x;           // [T, H]
-    const __half* residual;    // [T, H]
     const __half* gamma;       // [H]
     const __half* bias;        // [N] or null
     __half* residual_out;      // [T, H]
@@ -55,28 +70,24 @@ struct QkvParams {
     int32_t T, H, N;
     int32_t q_cols, kv_cols;   // Hq * D, Hkv * D
     int32_t kblocks;           // H / 64
-    int32_t split;             // slices of H per run = cluster size (<= kQkvMaxCluster)
-    int32_t slab_blocks;       // most 64-wide k blocks in one slice
-    int32_t ftiles;            // feature tiles of kFT rows covering N
-    int32_t tiles_per_cta;     // consecutive feature tiles one CTA streams
+    int32_t split;             // slices of H = cluster size (<= kQkvMaxCluster)
+    int32_t tt;                // tokens per tile: 64, 128 or 256
+    int32_t stages;            // ring depth (<= kQkvMaxStages)
     float eps;
     int32_t prefetch_w;        // request W tiles before the grid-dependency wait
 };
 
-template <int kMT, int kStages>
 struct QkvShape {
-    static constexpr int kFT = 128 * kMT;                 // features per tile (8 warps x 16 kMT)
-    static constexpr int kTT = 64;                        // tokens per CTA
-    static constexpr int kThreads = 256;
-    static constexpr int kStageBytes = kFT * 128;         // [kFT rows][64 k] f16
-    static constexpr int kHeader = 1024;                  // barriers and per-token values
-    static constexpr int kRedStride = kFT + 4;            // floats per token row of the partial tile
-    static constexpr int kRedBytes = kTT * kRedStride * 4;
-    static constexpr int kMaxSlabBytes = 232448 - 1024 - kHeader - kStages * kStageBytes - kRedBytes;
-    static constexpr int kMaxSlabBlocks = kMaxSlabBytes / (kTT * 128);
-    static_assert(kRedBytes % 1024 == 0, "the slab stays 1024-byte aligned");
-    static size_t smem_bytes(int slab_blocks) {
-        return 1024 + kHeader + (size_t)kStages * kStageBytes + kRedBytes + (size_t)kTT * slab_blocks * 128;
+    static constexpr int kThreads = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 scale + epilogue
+    static constexpr int kBuilders = 256;
+    static constexpr int kHeader = 4096;               // barriers and per-token values
+    static constexpr int kSmemMax = 232448 - 1024;     // the opt-in limit per block, less static room
+    __host__ __device__ static int stage_bytes(int m, int tt) { return m * 128 + tt * 128; }
+    __host__ __device__ static int gamma_bytes(int kblocks, int split) {   // the slice's gamma, 1024-aligned
+        return ((kblocks + split - 1) / split * 128 + 1023) & ~1023;
+    }
+    static size_t smem_bytes(int m, int tt, int stages, int kblocks, int split) {
+        return 1024 + kHeader + (size_t)gamma_bytes(kblocks, split) + (size_t)stages * stage_bytes(m, tt);
     }
 };
 
@@ -94,297 +105,306 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
                  :: "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// 2^n as a float for -126 <= n <= 127.
-__device__ __forceinline__ float exp2_int(int n) { return __int_as_float((127 + n) << 23); }
+// Barrier among the 256 build/epilogue threads only (named barrier 1).
+__device__ __forceinline__ void builders_sync() {
+    asm volatile("bar.sync 1, %0;" :: "n"(QkvShape::kBuilders) : "memory");
+}
 
-template <int kMT, int kStages>
-__global__ void __launch_bounds__(256, 1)
-add_rmsnorm_qkv_kernel(const __grid_constant__ CUtensorMap tm_w, const QkvParams p) {
-    using S = QkvShape<kMT, kStages>;
-    constexpr int kFT = S::kFT, kTT = S::kTT, kRS = S::kRedStride;
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ float sumsq_half2(uint32_t a, float acc) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&a));
+    return fmaf(f.y, f.y, fmaf(f.x, f.x, acc));
+}
+
+
+// s = f16(x + residual) into residual_out, 16 bytes per thread per step (the
+// first launch of the projection). `chunks` = T * H / 8.
+__global__ void __launch_bounds__(256)
+add_residual_kernel(const __half* __restrict__ x, const __half* __restrict__ residual, __half* __restrict__ out,
+                    int64_t chunks) {
+    grid_dependents_launch();                    // the projection may start requesting W tiles
+    grid_dependency_wait();                      // x and residual may come from the previous launch
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += stride) {
+        const uint4 a = ld_stream_16(reinterpret_cast<const uint4*>(x) + i);
+        const uint4 b = ld_stream_16(reinterpret_cast<const uint4*>(residual) + i);
+        uint4 r;
+        const __half2* a2 = reinterpret_cast<const __half2*>(&a);
+        const __half2* b2 = reinterpret_cast<const __half2*>(&b);
+        __half2* r2 = reinterpret_cast<__half2*>(&r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r2[e] = __hadd2(a2[e], b2[e]);   // one rounding, nearest even
+        reinterpret_cast<uint4*>(out)[i] = r;
+    }
+}
+
+template <int kAcc>   // 128-row halves of the W tile: M = 128 kAcc features
+__global__ void __launch_bounds__(QkvShape::kThreads, 1)
+rmsnorm_qkv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                   const QkvParams p) {
+    using S = QkvShape;
+    constexpr int kM = 128 * kAcc;
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-
     extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const base_ptr = smem_raw + (base - raw);
-    const uint32_t bars = base;                                           // kStages x 8 bytes
-    float* const ssq = reinterpret_cast<float*>(base_ptr + 64);           // [64] sum of s^2
-    float* const up = reinterpret_cast<float*>(base_ptr + 320);           // [64] 2^e_t
-    float* const rinv = reinterpret_cast<float*>(base_ptr + 576);         // [64] 1 / RMS
-    const uint32_t ring = base + S::kHeader;
-    float* const red = reinterpret_cast<float*>(base_ptr + S::kHeader + kStages * S::kStageBytes);
-    const uint32_t slab = ring + kStages * S::kStageBytes + S::kRedBytes;
-    const int slab_row = p.slab_blocks * 128;                             // bytes per token row
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int split = p.split;
+    const int split = p.split, TT = p.tt, NS = p.stages;
     const int rank = (int)cluster.block_rank();                           // == blockIdx.x % split
-    const int run = blockIdx.x / split;
-    const int ft0 = run * p.tiles_per_cta;                                // first feature tile of the run
-    const int nft = min(p.ftiles - ft0, p.tiles_per_cta);                 // >= 1
-    const int t0 = blockIdx.y * kTT;
+    const int m0 = (int)(blockIdx.x / split) * kM;                        // first feature of the tile
+    const int t0 = (int)blockIdx.y * TT;                                   // first token of the tile
     const int kb0 = (int)((int64_t)rank * p.kblocks / split);
-    const int nkb = (int)((int64_t)(rank + 1) * p.kblocks / split) - kb0; // >= 1: split <= kblocks
-    const int total = nft * nkb;                                          // W blocks this CTA streams
+    const int nkb = (int)((int64_t)(rank + 1) * p.kblocks / split) - kb0;  // >= 1: split <= kblocks
+
+    // ---- shared memory ----
+    const uint32_t bars = base;
+    auto full = [&](int s) { return bars + 8u * s; };                    // TMA landed (transaction bytes)
+    auto ready = [&](int s) { return bars + 64u + 8u * s; };             // W scaled (256 threads)
+    auto empty = [&](int s) { return bars + 128u + 8u * s; };            // the MMAs that read it are done
+    const uint32_t acc_full = bars + 192, tmem_slot = bars + 200;
+    float* const sqp = reinterpret_cast<float*>(base_ptr + 1024);         // [256]: per-thread sums of s^2
+    float* const sqt = reinterpret_cast<float*>(base_ptr + 2048);         // [TT]: over the slice, per token
+    float* const rinv = reinterpret_cast<float*>(base_ptr + 3072);        // [TT]: 1 / RMS of rank's tokens
+    const uint32_t gam = base + S::kHeader;                               // the slice's gamma [nkb][64]
+    const uint32_t ring = gam + S::gamma_bytes(p.kblocks, split);
+    const int stage = S::stage_bytes(kM, TT);
+    auto w_s = [&](int s) { return ring + (uint32_t)(s * stage); };
+    auto s_s = [&](int s) { return w_s(s) + kM * 128; };
+    float* const red = reinterpret_cast<float*>(base_ptr + (ring - base)); // [TT][kM] after the MMAs
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bars + 8 * s, 1);
+        s_abort = 0;
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(ready(s), S::kBuilders);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(acc_full, 1);
         mbar_init_fence();
     }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, (uint32_t)(kAcc * TT));
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    // W block i (feature tile i / nkb of the run, k block i % nkb of the slice)
-    // into slot i % kStages (thread 0)
-    auto issue = [&](int i) {
-        const int s = i % kStages;
-        const int j = i / nkb;
-        mbar_arrive_expect_tx(bars + 8 * s, S::kStageBytes);
-        tma_load_2d(ring + s * S::kStageBytes, &tm_w, bars + 8 * s, (kb0 + i - j * nkb) * 64, (ft0 + j) * kFT);
+    tc_fence_after();
+    uint32_t tmem;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_slot) : "memory");
+    grid_dependents_launch();
+
+    // Bounded wait that also gives up once another role has given up.
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (mbar_try_wait(bar, parity)) return true;
+        const uint64_t t_start = global_timer_ns();
+        for (uint32_t it = 0;; ++it) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if ((it & 63u) == 63u) {
+                if (*reinterpret_cast<volatile int*>(&s_abort)) return false;
+                if (global_timer_ns() - t_start > kWaitLimitNs) {
+                    flag_error(PKV_DEVERR_WAIT_TIMEOUT);
+                    *reinterpret_cast<volatile int*>(&s_abort) = 1;
+                    return false;
+                }
+            }
+        }
     };
-    const int prologue = min(total, kStages);
-    if (tid == 0) {
-        prefetch_tensormap(&tm_w);
-        if (p.prefetch_w)
-            for (int i = 0; i < prologue; ++i) issue(i);
-    }
-    grid_dependency_wait();
-    if (tid == 0 && !p.prefetch_w)
-        for (int i = 0; i < prologue; ++i) issue(i);
 
-    // ---- the slice's activations: warp w builds tokens w, w + 8, ..., w + 56 ----
-    {
-        const int cpt = nkb * 8;                  // 16-byte chunks per token row of the slice
-        const bool write_res = run == 0;
-        auto slab_addr = [&](int tl, int ch) {
-            return slab + tl * slab_row + (((ch & ~7) | ((ch ^ tl) & 7)) << 4);
-        };
-        // max |gamma| over the slice (every warp, the same value)
-        __half2 gm = __float2half2_rn(0.f);
-        for (int ch = lane; ch < cpt; ch += 32) {
-            const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma + (int64_t)kb0 * 64 + ch * 8));
-            const __half2* g2 = reinterpret_cast<const __half2*>(&gv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) gm = __hmax2(gm, __habs2(g2[e]));
+    bool ok = true;
+    if (warp == 0) {
+        // ================================ TMA ================================
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(&tm_s);
         }
-        float gmax = fmaxf(__low2float(gm), __high2float(gm));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
-
-        float sq[8];
-        __half2 mx[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            sq[j] = 0.f;
-            mx[j] = __float2half2_rn(0.f);
-        }
-        for (int ch = lane; ch < cpt; ch += 32) {
-            const int64_t kg = (int64_t)kb0 * 64 + ch * 8;
-            uint4 xv[8], rv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int t = t0 + warp + 8 * j;
-                if (t < p.T) {
-                    const int64_t off = (int64_t)t * p.H + kg;
-                    xv[j] = ld_stream_16(reinterpret_cast<const uint4*>(p.x + off));
-                    rv[j] = ld_stream_16(reinterpret_cast<const uint4*>(p.residual + off));
-                } else {
-                    xv[j] = rv[j] = make_uint4(0, 0, 0, 0);
-                }
+        const uint32_t tx = (uint32_t)stage;
+        const int pre = p.prefetch_w ? min(NS, nkb) : 0;
+        if (lane == 0)
+            for (int j = 0; j < pre; ++j) {
+                mbar_arrive_expect_tx(full(j), tx);
+                tma_load_2d(w_s(j), &tm_w, full(j), (kb0 + j) * 64, m0);
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int tl = warp + 8 * j;
-                uint4 sv;
-                __half2* s2 = reinterpret_cast<__half2*>(&sv);
-                const __half2* x2 = reinterpret_cast<const __half2*>(&xv[j]);
-                const __half2* r2 = reinterpret_cast<const __half2*>(&rv[j]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    s2[e] = __hadd2(x2[e], r2[e]);            // one rounding to f16, nearest even
-                    mx[j] = __hmax2(mx[j], __habs2(s2[e]));
-                    const float2 sf = __half22float2(s2[e]);
-                    sq[j] = fmaf(sf.x, sf.x, sq[j]);
-                    sq[j] = fmaf(sf.y, sf.y, sq[j]);
-                }
-                if (t0 + tl < p.T && write_res)
-                    *reinterpret_cast<uint4*>(p.residual_out + (int64_t)(t0 + tl) * p.H + kg) = sv;
-                sts128(slab_addr(tl, ch), sv);
-            }
-        }
-        // per token: the sum of squares, and the operand's power-of-two scale
-        float down[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float m = fmaxf(__low2float(mx[j]), __high2float(mx[j]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            }
-            const float bound = m * gmax;                 // >= max |s * gamma| over the slice
-            int e = 0;
-            if (bound > 0.f && bound <= 3.402823466e38f) {
-                const int E = (int)((__float_as_uint(bound) >> 23) & 0xFF) - 126;   // bound in [2^(E-1), 2^E)
-                e = E - 15;                                                           // bound * 2^-e in [2^14, 2^15)
-            }
-            down[j] = exp2_int(-e);
+        grid_dependency_wait();                                            // s is the first launch's output
+        if (lane == 0)
+            for (int j = 0; j < pre; ++j) tma_load_2d(s_s(j), &tm_s, full(j), (kb0 + j) * 64, t0);
+        int j = pre;
+        for (; j < nkb; ++j) {
+            const int s = j % NS;
+            if (j >= NS && !(ok = __all_sync(0xffffffffu, wait(empty(s), ((j / NS) - 1) & 1)))) break;
             if (lane == 0) {
-                ssq[warp + 8 * j] = sq[j];
-                up[warp + 8 * j] = exp2_int(e);
+                mbar_arrive_expect_tx(full(s), tx);
+                tma_load_2d(w_s(s), &tm_w, full(s), (kb0 + j) * 64, m0);
+                tma_load_2d(s_s(s), &tm_s, full(s), (kb0 + j) * 64, t0);
             }
         }
-        // b = f16(s * gamma * 2^-e): s * gamma is exact in fp32, the power of two too
-        for (int ch = lane; ch < cpt; ch += 32) {
-            const int64_t kg = (int64_t)kb0 * 64 + ch * 8;
-            const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma + kg));
-            const __half2* g2 = reinterpret_cast<const __half2*>(&gv);
-            float2 gf[4];
+        // nothing of ours may be in flight when the CTA leaves
+        for (int i = max(0, j - NS); i < j; ++i) mbar_wait(full(i % NS), (i / NS) & 1);
+    } else if (warp == 1) {
+        // ================================ MMA ================================
+        const uint32_t idesc = umma_idesc_f16(128, TT, 0);               // W' and s both K-major
+        for (int j = 0; j < nkb; ++j) {
+            const int s = j % NS;
+            if (!(ok = __all_sync(0xffffffffu, wait(ready(s), (j / NS) & 1)))) break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) gf[e] = __half22float2(g2[e]);
+                for (int a = 0; a < kAcc; ++a)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int tl = warp + 8 * j;
-                const uint32_t a = slab_addr(tl, ch);
-                uint4 sv = lds128(a), bv;
-                const __half2* s2 = reinterpret_cast<const __half2*>(&sv);
-                __half2* b2 = reinterpret_cast<__half2*>(&bv);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + (uint32_t)(a * TT), umma_desc_sw128(w_s(s) + a * 16384 + kk * 32, 16, 1024),
+                                    umma_desc_sw128(s_s(s) + kk * 32, 16, 1024), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(empty(s));
+            }
+            __syncwarp();
+        }
+        // completes once every MMA issued above has (also after a timeout)
+        if (lane == 0) umma_commit(acc_full);
+        __syncwarp();
+    } else {
+        // ========================= scale, then epilogue ========================
+        const int bt = tid - 64;                                           // 0 .. 255
+        const int nsub = S::kBuilders / TT;                                // threads per token: 4, 2 or 1
+        const int tok = bt % TT, sub = bt / TT, cpt = 8 / nsub;            // 16-byte chunks per k block
+        grid_dependency_wait();
+        // the slice's gamma, once
+        for (int i = bt; i < nkb * 8; i += S::kBuilders)
+            sts128(gam + 16 * i, __ldg(reinterpret_cast<const uint4*>(p.gamma + (int64_t)kb0 * 64) + i));
+        builders_sync();
+        float sq = 0.f;
+        for (int j = 0; j < nkb; ++j) {
+            const int s = j % NS;
+            if (!(ok = __all_sync(0xffffffffu, wait(full(s), (j / NS) & 1)))) break;
+            // this token's s^2 over this thread's chunks (logical chunk c sits at c ^ (row & 7))
+            for (int c = sub * cpt; c < sub * cpt + cpt; ++c) {
+                const uint4 sv = lds128(s_s(s) + (uint32_t)(tok * 128 + ((c ^ (tok & 7)) << 4)));
+                sq = sumsq_half2(sv.w, sumsq_half2(sv.z, sumsq_half2(sv.y, sumsq_half2(sv.x, sq))));
+            }
+            // W' = f16(W * gamma) on this thread's share of the tile's kM x 8 chunks
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 sf = __half22float2(s2[e]);
-                    b2[e] = __floats2half2_rn(sf.x * gf[e].x * down[j], sf.y * gf[e].y * down[j]);
+            for (int i = bt; i < kM * 8; i += S::kBuilders) {
+                const int row = i >> 3, c = i & 7;
+                const uint32_t off = (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
+                uint4 wv = lds128(w_s(s) + off);
+                const uint4 gv = lds128(gam + j * 128 + 16 * c);
+                wv.x = hmul2_u32(wv.x, gv.x);
+                wv.y = hmul2_u32(wv.y, gv.y);
+                wv.z = hmul2_u32(wv.z, gv.z);
+                wv.w = hmul2_u32(wv.w, gv.w);
+                sts128(w_s(s) + off, wv);
+            }
+            fence_proxy_async_shared();
+            mbar_arrive(ready(s));
+        }
+        sqp[sub * TT + tok] = sq;
+        if (ok) ok = __all_sync(0xffffffffu, wait(acc_full, 0));
+        tc_fence_after();
+        builders_sync();
+        if (bt < TT) {                                                     // the slice's sum, in sub order
+            float a = 0.f;
+            for (int u = 0; u < nsub; ++u) a += sqp[u * TT + bt];
+            sqt[bt] = a;
+        }
+        // the partial tile out of TMEM: red[token][feature] (every load landed, every MMA done)
+        if (ok) {
+            const int qd = warp & 3, hf = (warp - 2) >> 2;                 // TMEM lane quarter, column half
+#pragma unroll 1
+            for (int a = 0; a < kAcc; ++a) {
+                const int f = 128 * a + 32 * qd + lane;
+#pragma unroll 1
+                for (int c0 = hf * (TT / 2); c0 < (hf + 1) * (TT / 2); c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(a * TT + c0), v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) red[(c0 + i) * kM + f] = v[i];
                 }
-                sts128(a, bv);
             }
         }
+        tc_fence_before();
     }
-    __syncthreads();
 
-    const int lr = lane & 15, lh = lane >> 4;     // A: row within 16, k half
-    const int bm = lane >> 3, br = lane & 7;      // B: matrix of the x4 load, row within it
-    const int g = lane >> 2, c = lane & 3;        // accumulator: feature row, token pair
-    const int ta = rank * kTT / split, tb = (rank + 1) * kTT / split;   // this rank's tokens of a tile
-    bool failed = false;
-    int i = 0;                                    // W block counter over the run
-    for (int j = 0; j < nft; ++j) {
-        // ---- stream the tile's W blocks: 4 k16 steps per 64-wide block ----
-        float acc[kMT][8][4];
+    // ---- every rank's partial tile and sums of squares are in its shared memory ----
+    cluster.sync();
+    if (warp >= 2) {
+        const int bt = tid - 64;
+        const int tr0 = rank * TT / split, tr1 = (rank + 1) * TT / split;   // this rank's tokens of the tile
+        // 1 / RMS of those tokens: the ranks' sums of squares, all requested before any is added
+        for (int t = tr0 + bt; t < tr1; t += S::kBuilders) {
+            float u[kQkvMaxCluster];
 #pragma unroll
-        for (int mt = 0; mt < kMT; ++mt)
+            for (int r = 0; r < kQkvMaxCluster; ++r) u[r] = r < split ? *cluster.map_shared_rank(sqt + t, r) : 0.f;
+            float a = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-        for (int kk = 0; kk < nkb; ++kk, ++i) {
-            const int s = i % kStages;
-            const bool ok = !failed && mbar_wait(bars + 8 * s, (i / kStages) & 1);
-            if (ok) {
-                const uint32_t wt = ring + s * S::kStageBytes;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint32_t a[kMT][4];
-#pragma unroll
-                    for (int mt = 0; mt < kMT; ++mt) {
-                        const int row = (warp * kMT + mt) * 16 + lr;
-                        const int chunk = 2 * ks + lh;
-                        ldsm_x4(wt + row * 128 + ((chunk ^ (row & 7)) << 4), a[mt][0], a[mt][1], a[mt][2],
-                                a[mt][3]);
-                    }
-#pragma unroll
-                    for (int np = 0; np < 4; ++np) {     // two n8 token tiles per x4 load
-                        const int tl = np * 16 + (bm >> 1) * 8 + br;
-                        const int ch = kk * 8 + 2 * ks + (bm & 1);
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(slab + tl * slab_row + (((ch & ~7) | ((ch ^ tl) & 7)) << 4), b0, b1, b2, b3);
-#pragma unroll
-                        for (int mt = 0; mt < kMT; ++mt) {
-                            mma_16816(acc[mt][2 * np], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
-                            mma_16816(acc[mt][2 * np + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
-                        }
-                    }
-                }
-            }
-            // a lost TMA is flagged by mbar_wait; every thread then skips the rest of the
-            // stream but still takes every cluster barrier below
-            if (__syncthreads_or(!ok)) failed = true;
-            else if (tid == 0 && i + kStages < total) {
-                fence_proxy_async_shared();       // the slot's reads by ldmatrix come first
-                issue(i + kStages);
-            }
+            for (int r = 0; r < kQkvMaxCluster; ++r) a += u[r];             // rank order (the rest add 0)
+            rinv[t] = 1.f / sqrtf(a / (float)p.H + p.eps);
         }
-        if (j == nft - 1) grid_dependents_launch();
-
-        // ---- partial tile, scaled back by 2^e_t, as red[token][feature] ----
+        builders_sync();
+        // (token, 4 features) items, two at a time: the partial tiles summed in rank order, / RMS,
+        // + bias, f16; every remote load of both items is issued before the first sum
+        constexpr int kChunks = kM / 4;
+        const int items = (tr1 - tr0) * kChunks;
+        for (int i0 = bt; i0 < items; i0 += 2 * S::kBuilders) {
+            float4 u[2][kQkvMaxCluster];
 #pragma unroll
-        for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int f = (warp * kMT + mt) * 16 + g;
-                const int tk = nt * 8 + 2 * c;
-                const float u0 = up[tk], u1 = up[tk + 1];
-                red[tk * kRS + f] = acc[mt][nt][0] * u0;
-                red[(tk + 1) * kRS + f] = acc[mt][nt][1] * u1;
-                red[tk * kRS + f + 8] = acc[mt][nt][2] * u0;
-                red[(tk + 1) * kRS + f + 8] = acc[mt][nt][3] * u1;
-            }
-        cluster.sync();                           // every rank's partials (and sums of squares) are written
-
-        if (j == 0) {                             // 1 / RMS of this rank's tokens, for every tile
-            if (tid < tb - ta) {
-                const int tk = ta + tid;
-                float part[kQkvMaxCluster];
+            for (int h = 0; h < 2; ++h) {
+                const int it = min(i0 + h * S::kBuilders, items - 1);
+                const int t = tr0 + it / kChunks, fc = (it % kChunks) * 4;
 #pragma unroll
                 for (int r = 0; r < kQkvMaxCluster; ++r)
-                    part[r] = r < split ? *cluster.map_shared_rank(ssq + tk, r) : 0.f;
-                float tot = 0.f;
-#pragma unroll
-                for (int r = 0; r < kQkvMaxCluster; ++r) tot += part[r];
-                rinv[tk] = 1.0f / sqrtf(tot / (float)p.H + p.eps);
+                    u[h][r] = r < split ? *reinterpret_cast<const float4*>(cluster.map_shared_rank(red + t * kM + fc, r))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            __syncthreads();
-        }
-        // ---- rank r finishes tokens [ta, tb) of feature tile ft0 + j ----
-        constexpr int kQuads = kFT / 4;
-        const int f0 = (ft0 + j) * kFT;
-        for (int it = tid; it < (tb - ta) * kQuads; it += S::kThreads) {
-            const int tk = ta + it / kQuads, fq = (it % kQuads) * 4;
-            const int t = t0 + tk, n = f0 + fq;
-            if (t >= p.T || n >= p.N) continue;
-            float4 v[kQkvMaxCluster];
 #pragma unroll
-            for (int r = 0; r < kQkvMaxCluster; ++r)
-                if (r < split)
-                    v[r] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(red + tk * kRS + fq, r));
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int h = 0; h < 2; ++h) {
+                const int it = i0 + h * S::kBuilders;
+                if (it >= items) continue;
+                const int t = tr0 + it / kChunks, fc = (it % kChunks) * 4;
+                const int tg = t0 + t, n = m0 + fc;
+                if (tg >= p.T || n >= p.N) continue;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int r = 0; r < kQkvMaxCluster; ++r)
-                if (r < split) {
-                    sum.x += v[r].x;
-                    sum.y += v[r].y;
-                    sum.z += v[r].z;
-                    sum.w += v[r].w;
+                for (int r = 0; r < kQkvMaxCluster; ++r) {                 // rank order (the rest add 0)
+                    acc.x += u[h][r].x;
+                    acc.y += u[h][r].y;
+                    acc.z += u[h][r].z;
+                    acc.w += u[h][r].w;
                 }
-            const float ri = rinv[tk];
-            float o[4] = {sum.x * ri, sum.y * ri, sum.z * ri, sum.w * ri};
-            if (p.bias) {
-                const uint2 bv = __ldg(reinterpret_cast<const uint2*>(p.bias + n));
-                const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&bv.x));
-                const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&bv.y));
-                o[0] += b01.x;
-                o[1] += b01.y;
-                o[2] += b23.x;
-                o[3] += b23.y;
+                const float ri = rinv[t];
+                float2 b01 = make_float2(0.f, 0.f), b23 = b01;
+                if (p.bias) {
+                    const uint2 bv = __ldg(reinterpret_cast<const uint2*>(p.bias + n));
+                    b01 = __half22float2(*reinterpret_cast<const __half2*>(&bv.x));
+                    b23 = __half22float2(*reinterpret_cast<const __half2*>(&bv.y));
+                }
+                uint2 o;
+                o.x = pack_half2(acc.x * ri + b01.x, acc.y * ri + b01.y);
+                o.y = pack_half2(acc.z * ri + b23.x, acc.w * ri + b23.y);
+                __half* dst;
+                int64_t idx;
+                if (n < p.q_cols) {
+                    dst = p.q;
+                    idx = (int64_t)tg * p.q_cols + n;
+                } else if (n < p.q_cols + p.kv_cols) {
+                    dst = p.k;
+                    idx = (int64_t)tg * p.kv_cols + (n - p.q_cols);
+                } else {
+                    dst = p.v;
+                    idx = (int64_t)tg * p.kv_cols + (n - p.q_cols - p.kv_cols);
+                }
+                *reinterpret_cast<uint2*>(dst + idx) = o;
             }
-            __half* dst;
-            if (n < p.q_cols) dst = p.q + (int64_t)t * p.q_cols + n;
-            else if (n < p.q_cols + p.kv_cols) dst = p.k + (int64_t)t * p.kv_cols + (n - p.q_cols);
-            else dst = p.v + (int64_t)t * p.kv_cols + (n - p.q_cols - p.kv_cols);
-            uint2 ov;
-            ov.x = pack_half2(o[0], o[1]);
-            ov.y = pack_half2(o[2], o[3]);
-            *reinterpret_cast<uint2*>(dst) = ov;
         }
-        cluster.sync();                           // peers are done reading this CTA's partial tile
+    }
+    cluster.sync();                                      // peers are done reading this CTA's partial tile
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, (uint32_t)(kAcc * TT));
     }
 }
 
