@@ -26,8 +26,9 @@
 //  * The consumer warps' (m, l, O) are merged through shared memory. With one
 //    partition the CTA writes out[b, heads of g]; otherwise it writes the
 //    partition's (m, l, O/l) to the workspace and the CTA that finishes the
-//    last partition of (b, g) -- found by an atomic ticket, no waiting --
-//    merges all partitions by the log-sum-exp rule and writes the output.
+//    last partition of (b, g) -- found by a release-acquire ticket, no
+//    waiting -- merges all partitions by the log-sum-exp rule and writes the
+//    output, with 16 partitions' loads in flight per (head, 4 channels).
 //
 // FP8 E4M3 blocks are expanded to f16 in registers (exact), with k_scale
 // folded into the logit scale and v_scale into the output.
@@ -263,15 +264,16 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (nparts_b == 1) return;
 
     // ---- split-KV: the last partition of (b, g) to finish merges them all ----
-    __threadfence();
+    // The barrier orders every thread's workspace stores before thread 0's
+    // release-acquire ticket; the merger's loads follow its acquire and the
+    // barrier after it.
     consumer_sync(kCT);
     if (threadIdx.x == 0) {
-        const unsigned int prev = atomicAdd(p.ws_count + (int64_t)b * p.Hkv + g, 1u);
+        const unsigned int prev = atomic_add_acq_rel_gpu(p.ws_count + (int64_t)b * p.Hkv + g, 1u);
         s_is_last = prev == (unsigned int)(nparts_b - 1);
     }
     consumer_sync(kCT);
     if (!s_is_last) return;
-    __threadfence();
     // weights w_q = l_q * exp2(m_q - M) of every partition and head, staged in
     // shared memory (the ring is free), then one pass over the outputs
     float* wts = reinterpret_cast<float*>(ring_ptr);             // [G][nparts_b]
@@ -301,18 +303,32 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
             for (int q = lane; q < nparts_b; q += 32) wh[q] *= out_scale / sum;
         }
         consumer_sync(kCT);
-        for (int h = h_first; h < G; h += h_step) {
+        // one (head, 4 channels) item per thread, 16 partitions' float4 loads in flight at a time
+        constexpr int kBatch = 16;
+        for (int it = threadIdx.x; it < G * (kHeadDim / 4); it += kCT) {
+            const int h = it / (kHeadDim / 4), cq = it % (kHeadDim / 4);
             const float* wh = wts + h * nparts_b;
-            const float* src = p.ws_o + (row0 + h) * p.nparts * kHeadDim + d;
-            float acc = 0.f;
-            int q = 0;
-            for (; q + 4 <= nparts_b; q += 4) {
-                const float v0 = __ldcg(src + (q + 0) * kHeadDim), v1 = __ldcg(src + (q + 1) * kHeadDim);
-                const float v2 = __ldcg(src + (q + 2) * kHeadDim), v3 = __ldcg(src + (q + 3) * kHeadDim);
-                acc += wh[q] * v0 + wh[q + 1] * v1 + wh[q + 2] * v2 + wh[q + 3] * v3;
+            const float4* src = reinterpret_cast<const float4*>(p.ws_o + (row0 + h) * p.nparts * kHeadDim) + cq;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q0 = 0; q0 < nparts_b; q0 += kBatch) {
+                float4 v[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+                    if (q0 + u < nparts_b) v[u] = __ldcg(src + (int64_t)(q0 + u) * (kHeadDim / 4));
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+                    if (q0 + u < nparts_b) {                        // partition order
+                        const float w = wh[q0 + u];
+                        acc.x += w * v[u].x;
+                        acc.y += w * v[u].y;
+                        acc.z += w * v[u].z;
+                        acc.w += w * v[u].w;
+                    }
             }
-            for (; q < nparts_b; ++q) acc += wh[q] * __ldcg(src + q * kHeadDim);
-            out_g[h * kHeadDim + d] = __float2half_rn(acc);
+            uint2 o;
+            o.x = pack_half2(acc.x, acc.y);
+            o.y = pack_half2(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(out_g + h * kHeadDim + 4 * cq) = o;
         }
     } else {
         for (int h = h_first; h < G; h += h_step) {
