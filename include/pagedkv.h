@@ -140,8 +140,9 @@ pkv_status paged_kv_cache_write(const void* k_new, const void* v_new,
 /*
  * Bytes of workspace paged_gqa_decode_attention needs for these sizes:
  * 0 when partition_tokens == 0 (single pass); for partition_tokens > 0 the
- * partial results of ceil(max_context_len / partition_tokens) partitions per
- * (sequence, query head) plus one counter per (sequence, KV head); for
+ * partial results of n = ceil(max_context_len / partition_tokens) partitions
+ * per (sequence, query head) plus the counters of their merge tree (fan-in 8:
+ * one per partition per level, ceil(log8 n) levels, per (sequence, KV head)); for
  * PKV_PARTITION_AUTO two partial results per worker warp of the persistent
  * grid on the CURRENT device plus the counters. Returns 0 for invalid sizes.
  */

@@ -25,10 +25,11 @@
 //    stage with an arrive on its "empty" mbarrier.
 //  * The consumer warps' (m, l, O) are merged through shared memory. With one
 //    partition the CTA writes out[b, heads of g]; otherwise it writes the
-//    partition's (m, l, O/l) to the workspace and the CTA that finishes the
-//    last partition of (b, g) -- found by a release-acquire ticket, no
-//    waiting -- merges all partitions by the log-sum-exp rule and writes the
-//    output, with 16 partitions' loads in flight per (head, 4 channels).
+//    partition's (m, l, O/l) to the workspace, and the partitions of (b, g)
+//    merge by the log-sum-exp rule in a tree of fan-in 8: the CTA that
+//    finishes a group last (a release-acquire ticket, no waiting) merges its
+//    entries, every load in flight at once, into the group's first entry;
+//    the merge that leaves one entry writes the output.
 //
 // FP8 E4M3 blocks are expanded to f16 in registers (exact), with k_scale
 // folded into the logit scale and v_scale into the output.
@@ -46,7 +47,7 @@ struct DecodeParams {
     float* ws_o;                  // [B*Hq, nparts, D]   partition outputs O/l
     float* ws_m;                  // [B*Hq, nparts]      partition max (exp2 domain)
     float* ws_l;                  // [B*Hq, nparts]      partition sum
-    unsigned int* ws_count;       // [B*Hkv]             finished partitions (ticket)
+    unsigned int* ws_count;       // [levels][B*Hkv][nparts] merge-tree tickets, zero between calls
     int32_t Hq, Hkv, G;
     int32_t max_blocks_per_seq, num_blocks, max_context_len;
     int32_t partition_tokens;     // multiple of kPageRows
@@ -57,6 +58,17 @@ struct DecodeParams {
     const float* v_scales;        // logit scale is logit_scale_log2 * k_scales[g], the output v_scales[g]
     int32_t scales_per_head;
 };
+
+// Fan-in of the split-KV merge tree over fixed partitions: a merge reads at
+// most this many partition entries, all of them in flight at once.
+constexpr int kPartFan = 8;
+
+// Levels of that tree for n partitions (1 for n <= kPartFan).
+__host__ __device__ constexpr int part_merge_levels(int n) {
+    int l = 1;
+    for (int64_t c = kPartFan; c < n; c *= kPartFan) ++l;
+    return l;
+}
 
 template <bool kFp8, int kConsumers, int kStages>
 struct DecodeShape {
@@ -263,88 +275,83 @@ decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     if (nparts_b == 1) return;
 
-    // ---- split-KV: the last partition of (b, g) to finish merges them all ----
-    // The barrier orders every thread's workspace stores before thread 0's
-    // release-acquire ticket; the merger's loads follow its acquire and the
-    // barrier after it.
-    consumer_sync(kCT);
-    if (threadIdx.x == 0) {
-        const unsigned int prev = atomic_add_acq_rel_gpu(p.ws_count + (int64_t)b * p.Hkv + g, 1u);
-        s_is_last = prev == (unsigned int)(nparts_b - 1);
-    }
-    consumer_sync(kCT);
-    if (!s_is_last) return;
-    // weights w_q = l_q * exp2(m_q - M) of every partition and head, staged in
-    // shared memory (the ring is free), then one pass over the outputs
-    float* wts = reinterpret_cast<float*>(ring_ptr);             // [G][nparts_b]
-    const bool staged = (size_t)G * nparts_b * sizeof(float) <= (size_t)S::kRingBytes;
-    if (staged) {
-        for (int i = threadIdx.x; i < G * nparts_b; i += kCT) {
-            const int h = i / nparts_b, q = i - h * nparts_b;
-            wts[i] = __ldcg(p.ws_m + (row0 + h) * p.nparts + q);
+    // ---- split-KV: a merge tree of fan-in kPartFan over the partitions ----
+    // Level 0 items are the partitions. At each level the last item of a group
+    // of kPartFan to finish (a release-acquire ticket, no waiting) merges the
+    // group by the log-sum-exp rule into the entry of the group's first item;
+    // the merge that leaves one item writes the output.
+    const int64_t BH = (int64_t)gridDim.z * p.Hkv;
+    int item = part, n_items = nparts_b, span = 1;
+    for (int lvl = 0;; ++lvl) {
+        const int first = item - item % kPartFan, last = min(first + kPartFan, n_items) - 1;
+        unsigned int* cnt = p.ws_count + ((int64_t)lvl * BH + (int64_t)b * p.Hkv + g) * p.nparts + first * span;
+        // The barrier orders every thread's workspace stores before thread 0's
+        // ticket; the merger's loads follow its acquire and the barrier after it.
+        consumer_sync(kCT);
+        if (threadIdx.x == 0) {
+            const unsigned int prev = atomic_add_acq_rel_gpu(cnt, 1u);
+            s_is_last = prev == (unsigned int)(last - first);
         }
         consumer_sync(kCT);
-        // one warp per head: max, weights, normaliser
-        for (int h = warp; h < G; h += kConsumers) {
-            float* wh = wts + h * nparts_b;
-            float M = -INFINITY;
-            for (int q = lane; q < nparts_b; q += 32) M = fmaxf(M, wh[q]);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-            float sum = 0.f;
-            for (int q = lane; q < nparts_b; q += 32) {
-                const float w = __ldcg(p.ws_l + (row0 + h) * p.nparts + q) * fast_exp2(wh[q] - M);
-                wh[q] = w;
-                sum += w;
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            __syncwarp();
-            for (int q = lane; q < nparts_b; q += 32) wh[q] *= out_scale / sum;
-        }
-        consumer_sync(kCT);
-        // one (head, 4 channels) item per thread, 16 partitions' float4 loads in flight at a time
-        constexpr int kBatch = 16;
+        if (!s_is_last) return;
+        const int n_it = last - first + 1;
+        const int n_next = (n_items + kPartFan - 1) / kPartFan;
+        // one (head, 4 channels) item per thread; the items' (m, l) and O are requested together,
+        // one round trip, and weighted after they land (a warp serves one head)
         for (int it = threadIdx.x; it < G * (kHeadDim / 4); it += kCT) {
             const int h = it / (kHeadDim / 4), cq = it % (kHeadDim / 4);
-            const float* wh = wts + h * nparts_b;
-            const float4* src = reinterpret_cast<const float4*>(p.ws_o + (row0 + h) * p.nparts * kHeadDim) + cq;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int q0 = 0; q0 < nparts_b; q0 += kBatch) {
-                float4 v[kBatch];
+            const int64_t e0 = (row0 + h) * p.nparts + (int64_t)first * span;
+            float4* base = reinterpret_cast<float4*>(p.ws_o + e0 * kHeadDim) + cq;
+            float4 v[kPartFan];
+            float mj[kPartFan], lj[kPartFan];
 #pragma unroll
-                for (int u = 0; u < kBatch; ++u)
-                    if (q0 + u < nparts_b) v[u] = __ldcg(src + (int64_t)(q0 + u) * (kHeadDim / 4));
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u)
-                    if (q0 + u < nparts_b) {                        // partition order
-                        const float w = wh[q0 + u];
-                        acc.x += w * v[u].x;
-                        acc.y += w * v[u].y;
-                        acc.z += w * v[u].z;
-                        acc.w += w * v[u].w;
-                    }
-            }
-            uint2 o;
-            o.x = pack_half2(acc.x, acc.y);
-            o.y = pack_half2(acc.z, acc.w);
-            *reinterpret_cast<uint2*>(out_g + h * kHeadDim + 4 * cq) = o;
-        }
-    } else {
-        for (int h = h_first; h < G; h += h_step) {
-            const int64_t pr0 = (row0 + h) * p.nparts;
+            for (int j = 0; j < kPartFan; ++j)
+                if (j < n_it) {
+                    const int64_t off = (int64_t)j * span;
+                    v[j] = __ldcg(base + off * (kHeadDim / 4));
+                    mj[j] = __ldcg(p.ws_m + e0 + off);
+                    lj[j] = __ldcg(p.ws_l + e0 + off);
+                }
             float M = -INFINITY;
-            for (int q = 0; q < nparts_b; ++q) M = fmaxf(M, __ldcg(p.ws_m + pr0 + q));
-            float wsum = 0.f, acc = 0.f;
-            for (int q = 0; q < nparts_b; ++q) {
-                const float w = __ldcg(p.ws_l + pr0 + q) * fast_exp2(__ldcg(p.ws_m + pr0 + q) - M);
-                wsum += w;
-                acc += w * __ldcg(p.ws_o + (pr0 + q) * kHeadDim + d);
+#pragma unroll
+            for (int j = 0; j < kPartFan; ++j)
+                if (j < n_it) M = fmaxf(M, mj[j]);
+            float L = 0.f;
+#pragma unroll
+            for (int j = 0; j < kPartFan; ++j)
+                if (j < n_it) {
+                    mj[j] = lj[j] * fast_exp2(mj[j] - M);          // the item's weight
+                    L += mj[j];
+                }
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kPartFan; ++j)
+                if (j < n_it) {                                    // item order
+                    const float w = mj[j] / L;
+                    acc.x += w * v[j].x;
+                    acc.y += w * v[j].y;
+                    acc.z += w * v[j].z;
+                    acc.w += w * v[j].w;
+                }
+            if (n_next == 1) {
+                uint2 o;
+                o.x = pack_half2(acc.x * out_scale, acc.y * out_scale);
+                o.y = pack_half2(acc.z * out_scale, acc.w * out_scale);
+                *reinterpret_cast<uint2*>(out_g + h * kHeadDim + 4 * cq) = o;
+            } else {
+                base[0] = acc;                                     // the group is one item of the next level
+                if (cq == 0) {
+                    p.ws_m[e0] = M;
+                    p.ws_l[e0] = L;
+                }
             }
-            out_g[h * kHeadDim + d] = __float2half_rn(acc / wsum * out_scale);
         }
+        if (threadIdx.x == 0) *cnt = 0u;                         // ready for the next call
+        if (n_next == 1) return;
+        item = first / kPartFan;
+        n_items = n_next;
+        span *= kPartFan;
     }
-    if (threadIdx.x == 0) p.ws_count[(int64_t)b * p.Hkv + g] = 0u;   // ready for the next call
 }
 
 }  // namespace pkv

@@ -314,7 +314,7 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t npa
     w.m = w.o + align256(rows * kHeadDim * sizeof(float));
     w.l = w.m + align256(rows * sizeof(float));
     w.count = w.l + align256(rows * sizeof(float));
-    w.total = w.count + align256(B * Hkv * sizeof(unsigned int));
+    w.total = w.count + align256(pkv::part_merge_levels((int)nparts) * B * Hkv * nparts * sizeof(unsigned int));
     return w;
 }
 

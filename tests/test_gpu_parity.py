@@ -350,6 +350,31 @@ def test_auto_one_sequence_split_over_many_workers():
     assert_attention_close(host(r.attention(AUTO)), r.oracle(), "auto long")
 
 
+@pytest.mark.parametrize("kv_dtype", ["f16", "fp8"])
+@pytest.mark.parametrize("P", [16, 64, 512])
+def test_fixed_partitions_merge_tree(P, kv_dtype):
+    """One 32k-token sequence in 2048, 512 or 64 partitions: a merge tree of fan-in 8 with 4, 3 or
+    2 levels and ragged groups, beside short one-partition sequences. The same workspace serves a
+    second call (every ticket back at zero) with the same bytes."""
+    base = "skewed-split" if kv_dtype == "f16" else "fp8-e4m3"
+    w = W.with_sizes(W.WORKLOADS[base], B=3, num_blocks=4096, ctx=("skewed", 32768, 2, 1, 50))
+    r = _run(w, 16)
+    B, Hq, D = r.q.shape
+    n = pkv.paged_gqa_decode_workspace_size(B, Hq, w.Hkv, D, r.max_len, P)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        out = torch.full((B, Hq, D), float("nan"), dtype=torch.float16, device="cuda")
+        pkv.paged_gqa_decode_attention(out, r.q, r.k, r.v, r.bt, r.cl, max_context_len=r.max_len,
+                                       softmax_scale=float(r.x["softmax_scale"]), kv_dtype=r.kv_dtype,
+                                       k_scale=float(r.x["k_scale"]), v_scale=float(r.x["v_scale"]),
+                                       partition_tokens=P, workspace=ws)
+        outs.append(host(out))
+    assert_attention_close(outs[0], r.oracle(), f"tree P={P} {kv_dtype}")
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+    assert pkv.pkv_device_error() == 0
+
+
 def test_auto_fp8_batch_beyond_its_tables_falls_back():
     """4000 sequences: the FP8 balanced tables no longer fit in shared memory while the f16
     ones do, so FP8 runs fixed partitions inside the workspace sized for the automatic plan."""
