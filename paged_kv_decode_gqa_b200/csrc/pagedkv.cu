@@ -714,8 +714,8 @@ bool make_q_map(CUtensorMap* map, const void* q, int Hq, int total, int G, int t
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// f16 prefill on tcgen05: one CTA per (tile of 128 / G query tokens, KV head,
-// sequence), one CTA per SM (its shared memory).
+// f16 prefill on tcgen05: one CTA per (two tiles of 128 / G query tokens, KV
+// head, sequence), one CTA per SM (its shared memory and TMEM).
 pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
                              int max_query_len, int Hkv, int B, cudaStream_t stream) {
     using S = pkv::PrefillTcShape;
@@ -725,7 +725,8 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& m
     auto kernel = pkv::prefill_tc_kernel<0>;
     static unsigned long long done = 0;
     if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
-    const dim3 grid((unsigned)((max_query_len + tokens - 1) / tokens), (unsigned)Hkv, (unsigned)B);
+    const int per_cta = S::kQTiles * tokens;                     // queries per CTA: two tiles
+    const dim3 grid((unsigned)((max_query_len + per_cta - 1) / per_cta), (unsigned)Hkv, (unsigned)B);
     return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm, tokens) == cudaSuccess
                ? PKV_OK : PKV_ERR_CUDA;
 }
