@@ -714,8 +714,9 @@ bool make_q_map(CUtensorMap* map, const void* q, int Hq, int total, int G, int t
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// f16 prefill on tcgen05: one CTA per (two tiles of 128 / G query tokens, KV
-// head, sequence), one CTA per SM (its shared memory and TMEM).
+// f16 prefill on tcgen05: a persistent grid of one CTA per SM (its shared
+// memory and TMEM) over items of (two tiles of 128 / G query tokens, KV head,
+// sequence).
 pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
                              int max_query_len, int Hkv, int B, cudaStream_t stream) {
     using S = pkv::PrefillTcShape;
@@ -725,9 +726,18 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& m
     auto kernel = pkv::prefill_tc_kernel<0>;
     static unsigned long long done = 0;
     if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
-    const int per_cta = S::kQTiles * tokens;                     // queries per CTA: two tiles
-    const dim3 grid((unsigned)((max_query_len + per_cta - 1) / per_cta), (unsigned)Hkv, (unsigned)B);
-    return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm, tokens) == cudaSuccess
+    // persistent: one CTA per SM (or per item when there are fewer), items of two query tiles
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const int per_item = S::kQTiles * tokens;                    // queries per item: two tiles
+    const int q_groups = (max_query_len + per_item - 1) / per_item;
+    const int64_t items = (int64_t)q_groups * Hkv * B;
+    if (items > INT32_MAX / 2) return PKV_ERR_UNSUPPORTED;      // item indices are int in the kernel
+    const dim3 grid((unsigned)std::min<int64_t>(items, sms));
+    return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm, tokens, q_groups, B) ==
+                   cudaSuccess
                ? PKV_OK : PKV_ERR_CUDA;
 }
 
