@@ -399,16 +399,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const bool edge = t0 + S::kKvTok - 1 > it.pos0 + t * T;   // some entries past a row's position
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float x[32];
-                    tmem_ld32(s_row + 32 * c, x);
-                    if (edge) {
+                for (int h = 0; h < 2; ++h) {                    // two 32-column loads in flight at a time
+                    float x[2][32];
+                    tmem_ld32x2(s_row + 64 * h, x[0], s_row + 64 * h + 32, x[1]);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            mx[i & 3] = fmaxf(mx[i & 3], t0 + 32 * c + i <= prow ? x[i] : -INFINITY);
-                    } else {
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const int c = 2 * h + c2;
+                        if (edge) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+                            for (int i = 0; i < 32; ++i)
+                                mx[i & 3] = fmaxf(mx[i & 3], t0 + 32 * c + i <= prow ? x[c2][i] : -INFINITY);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[c2][i]);
+                        }
                     }
                 }
                 float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
@@ -440,11 +444,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     float w[32];
+                    float xx[2][32];
+                    tmem_ld32x2(s_row + 64 * h, xx[0], s_row + 64 * h + 32, xx[1]);
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
                         const int c = 2 * h + c2;
-                        float x[32];
-                        tmem_ld32(s_row + 32 * c, x);
+                        const float (&x)[32] = xx[c2];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             float e0 = fmaf(x[2 * i], sl, -m_new), e1 = fmaf(x[2 * i + 1], sl, -m_new);

@@ -137,3 +137,25 @@ def test_prefill_zero_scale_is_the_causal_mean():
     x["softmax_scale"] = np.float32(0.0)
     assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "zero scale")
     assert pkv.pkv_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["qwen2.5-7b", "qwen2.5-1.5b"])
+def test_prefill_more_items_than_ctas_sampled(name):
+    """The bench's case at full size: 8 sequences append 512 tokens each to 2048-token contexts.
+    At 7B heads that is 480 work items (two 18-token query tiles, KV head, sequence), at 1.5B heads
+    208, more than the 148 CTAs of the persistent grid, so CTAs run several items each and carry
+    their barrier phases, Q reloads and accumulators from one item to the next. Sampled query rows
+    are checked against the float64 oracle: query i of sequence b is decode attention at context
+    length L_b - n_b + i + 1 over the same block table."""
+    B, n_new, L = 8, 512, 2048
+    w, x, q, qs = _case(name, 12, [n_new] * B, B=B, num_blocks=B * L // 16 + 64, ctx=("fixed", (L,) * B))
+    got = _run(w, x, q, qs)
+    rng = np.random.default_rng(13)
+    rows = np.sort(np.concatenate([rng.choice(int(qs[-1]), 40, replace=False), [0, int(qs[-1]) - 1]]))
+    b_of = np.searchsorted(qs, rows, side="right") - 1
+    ctx = (x["context_lens"][b_of] - (qs[b_of + 1] - qs[b_of]) + (rows - qs[b_of]) + 1).astype(np.int32)
+    ref = oracle.paged_gqa_decode(q[rows], x["k_pool"], x["v_pool"], x["block_tables"][b_of], ctx,
+                                  float(x["softmax_scale"]))
+    assert_attention_close(got[rows], ref, f"{name} sampled rows of {int(qs[-1])}")
+    assert np.isfinite(got).all()
+    assert pkv.pkv_device_error() == 0
