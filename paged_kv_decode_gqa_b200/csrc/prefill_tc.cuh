@@ -439,8 +439,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 m_run = m_new;
                 // pass 2: probabilities exp2(s * sl - m_new) as f16 pairs (tokens 2 i, 2 i + 1 of a 64-token
                 // half), one fused multiply-add and the fp32 exp2, masked entries 0; the row sum adds
-                // exactly those f16 values. P overwrites the logits it came from: the pairs of tokens
-                // 64 h .. 64 h + 63 go to columns 32 h .. 32 h + 31 of S_t, which pass 2 has read.
+                // exactly those f16 values, in four independent partial sums. P overwrites the logits it
+                // came from: the pairs of tokens 64 h .. 64 h + 63 go to columns 32 h .. 32 h + 31 of
+                // S_t, which pass 2 has read.
+                float lt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     float w[32];
@@ -458,12 +460,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 e1 = t0 + 32 * c + 2 * i + 1 <= prow ? e1 : -INFINITY;
                             }
                             const uint32_t pw = pack_half2(fast_exp2(e0), fast_exp2(e1));
-                            l_run = add_f16_hi(add_f16_lo(l_run, pw), pw);
+                            lt[i & 3] = add_f16_hi(add_f16_lo(lt[i & 3], pw), pw);
                             w[16 * c2 + i] = __uint_as_float(pw);
                         }
                     }
                     tmem_st32(s_row + 32 * h, w);
                 }
+                l_run += (lt[0] + lt[1]) + (lt[2] + lt[3]);
                 tmem_wait_st();                                  // P and any rescaled O are in TMEM
                 tc_fence_before();
                 mbar_arrive(p_full(t));
