@@ -329,7 +329,20 @@ pkv_status fused_add_rmsnorm_qkv(const void* x, const void* residual, const void
  * A sequence whose lengths are inconsistent on the device (n_b > L_b,
  * L_b > max_context_len, n_b > max_query_len, rows outside [0,
  * total_queries)) is flagged (PKV_DEVERR_CONTEXT_LEN) and its rows are left
- * unwritten. No workspace; supported shapes as for decode.
+ * unwritten. Supported shapes as for decode.
+ *
+ * workspace (optional, f16 cache): NULL runs whole work items (two query
+ *   tiles of one KV head of one sequence over all their KV tiles) on a
+ *   persistent grid, costliest first. With a workspace of
+ *   paged_gqa_prefill_workspace_size(...) bytes, 256-byte aligned and
+ *   ZERO-FILLED before its first use, every CTA takes an equal share of all
+ *   KV tiles of all items; an item cut at a CTA boundary is computed in
+ *   pieces whose partial (max, sum, output) rows the piece that finishes last
+ *   merges by the log-sum-exp rule of paged_gqa_decode_attention. A call
+ *   that completes without a device error leaves the workspace ready for the
+ *   next one; after PKV_DEVERR_WAIT_TIMEOUT zero-fill it again. Calls that
+ *   share a workspace must not run concurrently. A workspace that is too
+ *   small or misaligned returns PKV_ERR_WORKSPACE. FP8 caches ignore it.
  */
 pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
                                        const int32_t* block_tables, const int32_t* context_lens,
@@ -337,7 +350,17 @@ pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_c
                                        int32_t max_query_len, int32_t num_q_heads, int32_t num_kv_heads,
                                        int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
                                        int32_t num_blocks, int32_t max_context_len, float softmax_scale,
-                                       int32_t kv_dtype, float k_scale, float v_scale, void* stream);
+                                       int32_t kv_dtype, float k_scale, float v_scale, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
+ * Bytes of workspace paged_gqa_prefill_attention's load-balanced schedule
+ * needs on the CURRENT device: two partial results (both 128-row query
+ * tiles, fp32 output rows plus max and sum) per SM, then the merge tickets.
+ * 0 for an FP8 cache (its kernel takes none) and for invalid sizes.
+ */
+size_t paged_gqa_prefill_workspace_size(int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t kv_dtype);
 
 /*
  * fused_add_rmsnorm_qkv_plan -- the launch plan fused_add_rmsnorm_qkv uses on

@@ -53,8 +53,9 @@ _SIGNATURES = {
     "fused_add_rmsnorm_qkv": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _f32,
                                ctypes.c_uint32, _P], ctypes.c_int),
     "fused_add_rmsnorm_qkv_plan": ([_i32, _i32, _i32, _i32, _i32, _P], ctypes.c_int),
+    "paged_gqa_prefill_workspace_size": ([_i32, _i32, _i32, _i32], _sz),
     "paged_gqa_prefill_attention": ([_P, _P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
-                                     _i32, _i32, _i32, _f32, _i32, _f32, _f32, _P], ctypes.c_int),
+                                     _i32, _i32, _i32, _f32, _i32, _f32, _f32, _P, _sz, _P], ctypes.c_int),
 }
 # The symbols include/pagedkv.h declares (checked by the CPU tests).
 EXPORTED = tuple(_SIGNATURES)
@@ -378,11 +379,19 @@ def fused_add_rmsnorm_qkv_plan(T, H, Hq, Hkv, D) -> dict:
     return dict(zip(("tile_rows", "slices", "token_tile", "ctas", "token_tiles"), list(plan)))
 
 
+def paged_gqa_prefill_workspace_size(num_q_heads, num_kv_heads, head_dim, kv_dtype="f16") -> int:
+    """Bytes of workspace for the load-balanced prefill schedule on the current device (0: none)."""
+    return int(load_library().paged_gqa_prefill_workspace_size(num_q_heads, num_kv_heads, head_dim,
+                                                                kv_dtype_code(kv_dtype)))
+
+
 def paged_gqa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start, *,
                                 max_query_len, max_context_len, softmax_scale, kv_dtype="f16",
-                                k_scale=1.0, v_scale=1.0, stream=None) -> None:
+                                k_scale=1.0, v_scale=1.0, workspace=None, stream=None) -> None:
     """Chunked prefill: query rows q [total, Hq, D] of each sequence (query_start [B+1] int32), the
-    last n_b tokens of its context, attending causally through the block tables; out [total, Hq, D]."""
+    last n_b tokens of its context, attending causally through the block tables; out [total, Hq, D].
+    With a zero-filled workspace of paged_gqa_prefill_workspace_size bytes the f16 kernel balances
+    its work over the SMs (items cut at CTA boundaries and merged); without one, whole items."""
     _dense("out", out, "float16")
     _dense("q", q, "float16")
     for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
@@ -395,8 +404,11 @@ def paged_gqa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_
     B = context_lens.shape[0]
     if out.shape != q.shape or query_start.shape[0] != B + 1:
         raise ValueError("shape mismatch")
+    if workspace is not None:
+        _dense("workspace", workspace, "uint8", "float32", "int32")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load_library().paged_gqa_prefill_attention(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
         B, total, int(max_query_len), Hq, Hkv, D, bs, block_tables.shape[1], NB, int(max_context_len),
-        float(softmax_scale), kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _stream(stream)),
-        "paged_gqa_prefill_attention")
+        float(softmax_scale), kv_dtype_code(kv_dtype), float(k_scale), float(v_scale), _ptr(workspace), ws_bytes,
+        _stream(stream)), "paged_gqa_prefill_attention")

@@ -717,15 +717,31 @@ bool make_q_map(CUtensorMap* map, const void* q, int Hq, int total, int G, int t
 // f16 prefill on tcgen05: a persistent grid of one CTA per SM (its shared
 // memory and TMEM) over items of (two tiles of 128 / G query tokens, KV head,
 // sequence).
+// Workspace of the stream-K prefill schedule for a device of `ctas` SMs (grids of up to one CTA
+// per SM): two partial results (both query tiles) per CTA, then one ticket per (CTA, query tile,
+// row quarter).
+struct PrefillWorkspace {
+    int64_t parts, counters, total;
+};
+PrefillWorkspace prefill_layout(int64_t ctas) {
+    using S = pkv::PrefillTcShape;
+    PrefillWorkspace w;
+    w.parts = 0;
+    w.counters = 2 * ctas * S::kQTiles * (int64_t)S::kPartBytes;
+    w.total = (int64_t)align256((size_t)(w.counters + ctas * S::kQTiles * 4 * (int64_t)sizeof(unsigned int)));
+    return w;
+}
+
 pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
-                             int max_query_len, int Hkv, int B, cudaStream_t stream) {
+                             int max_query_len, int Hkv, int B, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
     using S = pkv::PrefillTcShape;
     const int tokens = S::kRows / prm.G;
     CUtensorMap mq;
     if (!make_q_map(&mq, prm.q, prm.Hq, prm.total, prm.G, tokens)) return PKV_ERR_CUDA;
-    auto kernel = pkv::prefill_tc_kernel<0>;
-    static unsigned long long done = 0;
-    if (ensure_smem(kernel, S::kSmemBytes, &done) != cudaSuccess) return PKV_ERR_CUDA;
+    auto kernel = workspace ? pkv::prefill_tc_kernel<true> : pkv::prefill_tc_kernel<false>;
+    static unsigned long long done[2] = {0, 0};
+    if (ensure_smem(kernel, S::kSmemBytes, &done[workspace ? 1 : 0]) != cudaSuccess) return PKV_ERR_CUDA;
     // persistent: one CTA per SM (or per item when there are fewer), items of two query tiles
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -735,9 +751,19 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& m
     const int q_groups = (max_query_len + per_item - 1) / per_item;
     const int64_t items = (int64_t)q_groups * Hkv * B;
     if (items > INT32_MAX / 2) return PKV_ERR_UNSUPPORTED;      // item indices are int in the kernel
-    const dim3 grid((unsigned)std::min<int64_t>(items, sms));
-    return launch_pdl(kernel, grid, dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm, tokens, q_groups, B) ==
-                   cudaSuccess
+    const int ctas = (int)std::min<int64_t>(items, sms);
+    uint8_t* ws = nullptr;
+    unsigned int* counters = nullptr;
+    if (workspace) {
+        // laid out for the device (not this call's grid), so that calls of any size can share it
+        const PrefillWorkspace w = prefill_layout(sms);
+        if (workspace_bytes < (size_t)w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return PKV_ERR_WORKSPACE;
+        ws = static_cast<uint8_t*>(workspace) + w.parts;
+        counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + w.counters);
+    }
+    return launch_pdl(kernel, dim3((unsigned)ctas), dim3(S::kThreads), S::kSmemBytes, stream, mq, mk, mv, prm,
+                      tokens, q_groups, B, ws, counters) == cudaSuccess
                ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -935,13 +961,27 @@ pkv_status paged_gqa_decode_step_fp8_scaled(
                      workspace, workspace_bytes, flags, stream);
 }
 
+size_t paged_gqa_prefill_workspace_size(int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t kv_dtype) {
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim || num_q_heads % num_kv_heads != 0 ||
+        num_q_heads / num_kv_heads > pkv::kGroupPad || (kv_dtype != PKV_KV_F16 && kv_dtype != PKV_KV_FP8_E4M3))
+        return 0;
+    if (kv_dtype == PKV_KV_FP8_E4M3) return 0;                  // the warp-level FP8 kernel takes none
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return 0;
+    return (size_t)prefill_layout(sms).total;
+}
+
 pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
                                        const int32_t* block_tables, const int32_t* context_lens,
                                        const int32_t* query_start, int32_t batch, int32_t total_queries,
                                        int32_t max_query_len, int32_t num_q_heads, int32_t num_kv_heads,
                                        int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
                                        int32_t num_blocks, int32_t max_context_len, float softmax_scale,
-                                       int32_t kv_dtype, float k_scale, float v_scale, void* stream) {
+                                       int32_t kv_dtype, float k_scale, float v_scale, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
     if (total_queries < 0 || max_query_len < 0) return PKV_ERR_INVALID_ARG;
     const bool any = batch > 0 && total_queries > 0 && max_query_len > 0;
     {
@@ -975,7 +1015,8 @@ pkv_status paged_gqa_prefill_attention(void* out, const void* q, const void* k_c
         !cached_cache_map(&mv, v_cache, fp8, num_blocks, num_kv_heads))
         return PKV_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (!fp8) return launch_prefill_tc(prm, mk, mv, max_query_len, num_kv_heads, batch, st);
+    if (!fp8)
+        return launch_prefill_tc(prm, mk, mv, max_query_len, num_kv_heads, batch, workspace, workspace_bytes, st);
     // an FP8 cache stays on the warp-level path: tcgen05 kind::f16 takes f16 operands only,
     // and an E4M3 query would not meet the attention tolerance
     const int chunks = (max_query_len + kPrefillConsumers - 1) / kPrefillConsumers;

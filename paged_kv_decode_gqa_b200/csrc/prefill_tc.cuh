@@ -10,48 +10,40 @@
 //
 // Unlike decode, prefill is a dense contraction, so each CTA runs it as two
 // GEMMs per KV tile on tcgen05:
-//  * Work unit: one CTA per (tile of T = floor(128 / G) query tokens, KV head
-//    g, sequence b). The tile's M = T * G <= 128 rows are its queries x the G
-//    query heads of g, row r = token r / G, head r % G, so every K/V byte a
-//    CTA stages serves all G heads of every query in it.
-//  * A KV tile is 128 tokens (8 pages). K and V pages come by TMA into
-//    three-stage rings, K and V with their own barriers and their own TMA
-//    warp: a K stage is refilled as soon as S of its tile is done, a V stage
-//    once O += P V of its tile is. Each refill takes over a microsecond to
-//    land from L2, so the rings hold as many tiles as shared memory allows:
-//    the probabilities stay in TMEM, which frees the room. Q (the CTA's rows)
-//    comes once.
-//  * The KV tiles are split by parity into two independent online softmaxes,
-//    each with its own running maximum, row sum and accumulator, merged by
-//    the log-sum-exp rule at the end (split-KV inside the CTA). Softmax warps
-//    0-3 serve the even tiles and warps 4-7 the odd ones; warps w and w + 4
-//    share a scheduler and a TMEM lane quarter (rows 32 (w % 4) .. +31), and
-//    as they work on different tiles one's exp2 runs while the other loads or
-//    takes maxima. A thread owns a whole row of its tiles, so no maximum
-//    crosses warps.
-//  * One thread issues S = Q K^T (M = 128, N = 128, K = 128; K-major A and
-//    B) into the TMEM columns of the tile's parity, [0, 128) or [128, 256),
-//    and after the softmax O_par += P V into [256, 384) or [384, 512), with P
+//  * Query tile: T = floor(128 / G) query tokens of one sequence x the G
+//    query heads of one KV head g, M = T * G <= 128 rows, row r = (token
+//    r / G, head r % G), so every K/V byte a CTA stages serves all G heads of
+//    every query in it. A work item is two such tiles (A and B, 2 T
+//    consecutive queries) of one (sequence, KV head), over the KV tiles
+//    their positions reach.
+//  * Persistent grid, one CTA per SM, TMEM, barriers and rings set up once;
+//    barrier phases run on across a CTA's work through global KV-tile and
+//    item counters. Without a workspace a CTA takes whole items, costliest
+//    first, in snake order. With one, every CTA takes an equal run of all
+//    items' KV tiles (stream-K); an item cut at a CTA boundary is computed
+//    in pieces, each piece stores its rows' (max, sum, unnormalised output),
+//    and the piece that takes the last ticket merges them by the log-sum-exp
+//    rule. Nobody waits on another CTA.
+//  * A KV tile is 128 tokens (8 pages). K and V have their own two-stage
+//    rings, barriers and TMA warp (warp 8: Q and K, warp 9: V). Pages past
+//    the item's last position are loaded from block -1, a box wholly outside
+//    the pool, which TMA fills with zeros; rows past the context in the
+//    sequence's last page are zeroed in shared memory before their V is used.
+//  * TMEM: S_A, S_B, O_A, O_B, 128 columns each. One thread (warp 10) issues
+//    S_t = Q_t K^T (M = N = K = 128, both K-major) and O_t += P_t V with P_t
 //    read from TMEM (the A operand of `tcgen05.mma` may live there: row r in
-//    lane r, two f16 per column) and V MN-major from shared memory. S of tile
-//    j + 1 is issued before O += P V of tile j; S of tile j + 2 waits until
-//    O += P V of tile j has read P out of the same columns.
-//  * Softmax of a tile, per thread (row r): pass 1 reads the row's 128
-//    logits from TMEM in four 32-column loads and takes their maximum (the
-//    causal mask only on tiles that reach past the tile's first position);
-//    the running maximum (exp2 domain) is raised only when a tile's maximum
-//    exceeds it by more than 8 (a factor 256), and only then are the row's
-//    accumulator and sum rescaled. Pass 2 reads the logits again and forms
-//    exp2(s * scale - m) with one fused multiply-add and the fp32 exp2,
-//    rounds to f16, adds exactly those f16 values to the row sum in fp32
-//    (mixed-precision add), and stores the f16 pairs over the logits already
-//    read. The output is (O_even a_e + O_odd a_o) / (l_e a_e + l_o a_o) in
-//    f16, a = exp2(m - max(m_e, m_o)); warps 0-3 write channels 0-63, 4-7
-//    the rest.
-//  * Rows past the context in the sequence's last page (free slots, any
-//    content) are zeroed in shared memory before their V is used; pages past
-//    the tile's last position are loaded from outside the pool, which TMA
-//    fills with zeros.
+//    lane r, two f16 per column) and V MN-major from shared memory. Per KV
+//    tile j: O_A += P_A V(j), S_A(j + 1), O_B += P_B V(j), S_B(j + 1), so the
+//    tensor core works on one tile while the other tile's softmax runs.
+//  * Softmax: warps 0-3 serve tile A, warps 4-7 tile B, one row (TMEM lane)
+//    per thread. Pass 1 takes the row's maximum (the causal mask only on KV
+//    tiles that reach past the query tile's first position); the running
+//    maximum (exp2 domain) is raised only when a tile's maximum exceeds it by
+//    more than 8 (a factor 256), and only then are the row's O and sum
+//    rescaled. Pass 2 forms exp2(s * scale - m) with one fused multiply-add
+//    and the fp32 exp2, rounds to f16, adds exactly those f16 values to the
+//    row sum in fp32 (mixed-precision add), and stores the f16 pairs over
+//    the logits already read. The output is O / sum in f16.
 // Every barrier wait has a time limit; one that runs out flags
 // PKV_DEVERR_WAIT_TIMEOUT and makes every role stop, wait for what it has in
 // flight, and leave; TMEM is always freed.
@@ -78,6 +70,10 @@ struct PrefillTcShape {
     static constexpr int kTmaKWarp = kSoftmaxWarps, kTmaVWarp = kSoftmaxWarps + 1, kMmaWarp = kSoftmaxWarps + 2;
     static constexpr uint32_t kTmemCols = 512;         // S_A, S_B (P over them), O_A, O_B: 128 columns each
     static constexpr float kRescaleThreshold = 8.f;    // log2 of the largest unnormalised probability
+    // stream-K schedule: one piece's partial result for one query tile, O as [32 float4 of
+    // channels][128 rows] and (m, l) per row; two slots per CTA (its first and its last piece)
+    static constexpr int kPartBytes = 128 * 128 * 4 + 128 * 8;
+    static constexpr int kMinTiles = 4;                // fewest KV tiles a CTA is given
 };
 
 // acc += the f16 value in the low (hi = false) or high half of w, exactly (mixed-precision add).
@@ -95,50 +91,193 @@ struct PrefillItem {
     int b, g, qs0, i0, nq, pos0, ntiles, npages, L;
 };
 
-template <int kDummy = 0>
+// The KV tiles [j0, j1) of an item that one CTA processes: the whole item, or a piece of it
+// when the stream-K schedule cuts the item at a CTA boundary. u: the item's first unit.
+struct PrefillPiece {
+    PrefillItem it;
+    int j0, j1;
+    int64_t u;
+};
+
+template <bool kStream>
 __global__ void __launch_bounds__(PrefillTcShape::kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p, const int tok_per_tile,
-                  const int q_groups, const int batch) {
+                  const int q_groups, const int batch, uint8_t* const ws, unsigned int* const ws_count) {
     using S = PrefillTcShape;
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
+    __shared__ long long s_red[S::kThreads / 32];
+    __shared__ long long s_first[2];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G, T = tok_per_tile;
 
     grid_dependency_wait();                      // inputs may come from the previous launch
     grid_dependents_launch();
-    // ---- work items: (group of two query tiles, KV head, sequence), costliest groups first ----
-    const int per_q = p.Hkv * batch;
-    const int n_items = q_groups * per_q;
-    const int C = gridDim.x;
-    // the r-th item of this CTA in the snake order (CTA c takes c, 2C - 1 - c, 2C + c, ...), or -1
-    auto item_index = [&](int r) -> int {
-        const int i = r * C + ((r & 1) ? C - 1 - (int)blockIdx.x : (int)blockIdx.x);
-        return i < n_items ? i : -1;
-    };
+    // ---- work items: (group of two query tiles, KV head, sequence) ----
     const int cap = min(p.max_context_len, p.max_blocks_per_seq * kPageRows);
-    // false: the item has no queries (or its sequence is inconsistent: flagged once, rows left alone)
-    auto item_info = [&](int i, PrefillItem& it) -> bool {
-        const int qg = q_groups - 1 - i / per_q, rem = i % per_q;
-        it.g = rem % p.Hkv;
-        it.b = rem / p.Hkv;
-        it.qs0 = __ldg(p.query_start + it.b);
-        const int qs1 = __ldg(p.query_start + it.b + 1);
-        it.L = __ldg(p.context_lens + it.b);
+    // item (query group qg, KV head g, sequence b): 1, or 0 when the group is past the
+    // sequence's queries, -1 when the sequence's lengths are inconsistent
+    auto make_item = [&](int b, int g, int qg, PrefillItem& it) -> int {
+        it.b = b;
+        it.g = g;
+        it.qs0 = __ldg(p.query_start + b);
+        const int qs1 = __ldg(p.query_start + b + 1);
+        it.L = __ldg(p.context_lens + b);
         const int n = qs1 - it.qs0;
-        if (it.qs0 < 0 || n < 0 || qs1 > p.total || n > p.max_query_len || it.L < n || it.L > cap) {
-            if (threadIdx.x == 0 && qg == 0 && it.g == 0) flag_error(PKV_DEVERR_CONTEXT_LEN);
-            return false;
-        }
+        if (it.qs0 < 0 || n < 0 || qs1 > p.total || n > p.max_query_len || it.L < n || it.L > cap) return -1;
         it.i0 = qg * S::kQTiles * T;             // first query of the item's two tiles
-        if (it.i0 >= n) return false;
+        if (it.i0 >= n) return 0;
         it.nq = min(S::kQTiles * T, n - it.i0);  // queries of the two tiles
         it.pos0 = it.L - n + it.i0;              // position of the first query
         const int p_max = it.pos0 + it.nq - 1;   // and of the last
         it.ntiles = p_max / S::kKvTok + 1;
         it.npages = p_max / kPageRows + 1;       // pages 0 .. npages-1 are read
-        return true;
+        return 1;
+    };
+    // Without a workspace every CTA takes whole items, costliest first (the last query groups
+    // see the longest contexts), dealt out in snake order: CTA c takes items c, 2C - 1 - c,
+    // 2C + c, ... of the C CTAs. With one (stream-K), the items in (sequence, KV head, query
+    // group) order form a row of U KV tiles ("units"); CTA c < C' takes units
+    // [c U / C', (c + 1) U / C'), C' <= C being the most CTAs that get kMinTiles or more, and
+    // an item cut at a CTA boundary becomes pieces whose partial softmaxes the piece that
+    // finishes last merges by the log-sum-exp rule.
+    constexpr bool stream = kStream;             // the launch passes a workspace exactly then
+    const int C = gridDim.x;
+    int64_t U = 0, u_lo = 0, u_hi = 0;
+    int ctas = 1;
+    // KV tiles of all items of sequence b under one KV head (0: no queries, or inconsistent)
+    auto seq_tiles = [&](int b) -> int64_t {
+        const int qs0 = __ldg(p.query_start + b), qs1 = __ldg(p.query_start + b + 1);
+        const int L = __ldg(p.context_lens + b), n = qs1 - qs0;
+        if (qs0 < 0 || n < 0 || qs1 > p.total || n > p.max_query_len || L < n || L > cap) return 0;
+        int64_t s = 0;
+        for (int i0 = 0; i0 < n; i0 += S::kQTiles * T) s += (L - n + min(i0 + S::kQTiles * T, n) - 1) / S::kKvTok + 1;
+        return s;
+    };
+    // inclusive scan of x over the block; total: the block's sum (uses s_red, ends synchronised)
+    auto block_scan = [&](int64_t x, int64_t& total) -> int64_t {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (lane == 31) s_red[warp] = x;
+        __syncthreads();
+        int64_t before = 0;
+        total = 0;
+        for (int i = 0; i < S::kThreads / 32; ++i) {
+            before += i < warp ? s_red[i] : 0;
+            total += s_red[i];
+        }
+        __syncthreads();
+        return before + x;
+    };
+    if (stream) {
+        // units of every sequence (all KV heads), scanned; the first chunk of sequences is kept
+        int64_t my_w = 0, my_incl = 0, first_total = 0;
+        for (int b0 = 0; b0 < batch; b0 += S::kThreads) {
+            const int b = b0 + (int)threadIdx.x;
+            int64_t w = 0;
+            if (b < batch) {
+                w = seq_tiles(b) * p.Hkv;
+                PrefillItem it;
+                if (blockIdx.x == 0 && make_item(b, 0, 0, it) < 0) flag_error(PKV_DEVERR_CONTEXT_LEN);
+            }
+            int64_t total;
+            const int64_t incl = U + block_scan(w, total);
+            if (b0 == 0) {
+                my_w = w;
+                my_incl = incl;
+                first_total = total;
+            }
+            U += total;
+        }
+        ctas = (int)max((int64_t)1, min((int64_t)C, U / S::kMinTiles));
+        u_lo = blockIdx.x < ctas ? (int64_t)blockIdx.x * U / ctas : U;
+        u_hi = blockIdx.x < ctas ? ((int64_t)blockIdx.x + 1) * U / ctas : U;
+        // the sequence that holds unit u_lo, and the units before it: in the first chunk from the
+        // values kept, past it (more sequences than threads) by scanning again
+        if (u_lo < u_hi) {
+            if (my_w > 0 && my_incl - my_w <= u_lo && u_lo < my_incl) {
+                s_first[0] = threadIdx.x;
+                s_first[1] = my_incl - my_w;
+            }
+            int64_t base = first_total;
+            for (int b0 = S::kThreads; b0 < batch && base <= u_lo; b0 += S::kThreads) {
+                const int b = b0 + (int)threadIdx.x;
+                const int64_t w = b < batch ? seq_tiles(b) * p.Hkv : 0;
+                int64_t total;
+                const int64_t incl = base + block_scan(w, total);
+                if (w > 0 && incl - w <= u_lo && u_lo < incl) {
+                    s_first[0] = b;
+                    s_first[1] = incl - w;
+                }
+                base += total;
+            }
+        }
+        __syncthreads();
+    }
+    // first unit of CTA c's range, and the CTA whose range holds unit u
+    auto range_lo = [&](int c) -> int64_t { return (int64_t)c * U / ctas; };
+    auto cta_of = [&](int64_t u) -> int {
+        int c = (int)min((int64_t)ctas - 1, u * ctas / U);
+        while (c > 0 && range_lo(c) > u) --c;
+        while (c + 1 < ctas && range_lo(c + 1) <= u) ++c;
+        return c;
+    };
+    // cursor: snake rank, or the stream-K item (qg of KV head cg of sequence cb, first unit cu)
+    int ri = 0, cb = batch, cg = 0, cq = 0;
+    int64_t cu = U;
+    if (stream && u_lo < u_hi) {
+        cb = (int)s_first[0];
+        const int64_t per_g = seq_tiles(cb);
+        cg = (int)((u_lo - s_first[1]) / per_g);
+        cu = s_first[1] + cg * per_g;
+        PrefillItem it;
+        while (make_item(cb, cg, cq, it) > 0 && cu + it.ntiles <= u_lo) {
+            cu += it.ntiles;
+            ++cq;
+        }
+    }
+    const int per_q = p.Hkv * batch;
+    const int n_items = q_groups * per_q;
+    // the CTA's next piece; false when it has none left
+    auto next_piece = [&](PrefillPiece& pc) -> bool {
+        if (!stream) {
+            for (;;) {
+                const int i = ri * C + ((ri & 1) ? C - 1 - (int)blockIdx.x : (int)blockIdx.x);
+                ++ri;
+                if (i >= n_items) return false;
+                const int qg = q_groups - 1 - i / per_q, rem = i % per_q;
+                const int r = make_item(rem / p.Hkv, rem % p.Hkv, qg, pc.it);
+                if (r < 0 && threadIdx.x == 0 && qg == 0 && rem % p.Hkv == 0) flag_error(PKV_DEVERR_CONTEXT_LEN);
+                if (r > 0) {
+                    pc.j0 = 0;
+                    pc.j1 = pc.it.ntiles;
+                    pc.u = 0;
+                    return true;
+                }
+            }
+        }
+        while (cu < u_hi && cb < batch) {
+            const int r = make_item(cb, cg, cq, pc.it);
+            if (r <= 0) {                        // next KV head, or next sequence
+                cq = 0;
+                if (r < 0 || ++cg == p.Hkv) {
+                    cg = 0;
+                    ++cb;
+                }
+                continue;
+            }
+            pc.u = cu;
+            pc.j0 = (int)(max(cu, u_lo) - cu);
+            pc.j1 = (int)(min(cu + pc.it.ntiles, u_hi) - cu);
+            cu += pc.it.ntiles;
+            ++cq;
+            return true;
+        }
+        return false;
     };
 
     // ---- shared memory ----
@@ -232,11 +371,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const CUtensorMap* map = is_k ? &tm_k : &tm_v;
         int gj = 0, k = 0;
         bool ok = true;
-        for (int ri = 0; ok; ++ri) {
-            const int item = item_index(ri);
-            if (item < 0) break;
-            PrefillItem it;
-            if (!item_info(item, it)) continue;
+        PrefillPiece pc;
+        while (ok && next_piece(pc)) {
+            const PrefillItem& it = pc.it;
             if (is_k) {
                 if (k >= 1 && !(ok = __all_sync(0xffffffffu, wait(q_empty, (k - 1) & 1)))) break;
                 if (lane == 0) {
@@ -249,7 +386,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             ++k;
             const int32_t* bt = p.block_tables + (int64_t)it.b * p.max_blocks_per_seq;
-            for (int j = 0; j < it.ntiles; ++j, ++gj) {
+            for (int j = pc.j0; j < pc.j1; ++j, ++gj) {
                 const int s = gj % S::kStages;
                 const uint32_t full = is_k ? k_full(s) : v_full(s), dst = is_k ? k_s(s) : v_s(s);
                 if (gj >= S::kStages &&
@@ -326,24 +463,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         };
         int gj = 0, k = 0;
         bool ok = true;
-        for (int ri = 0; ok; ++ri) {
-            const int item = item_index(ri);
-            if (item < 0) break;
-            PrefillItem it;
-            if (!item_info(item, it)) continue;
-            const int last_page = (it.L - 1) / kPageRows;
-            const int valid_last = it.L - last_page * kPageRows;     // live rows of that page
+        PrefillPiece pc;
+        while (ok && next_piece(pc)) {
+            // the piece's bounds and page limits, held in registers for the issue loop (the empty
+            // asm keeps the compiler from re-deriving them from the loads they came from in every
+            // iteration, which slowed each KV tile by about a tenth)
+            int pj0 = pc.j0, pj1 = pc.j1, npages = pc.it.npages;
+            int last_page = (pc.it.L - 1) / kPageRows;
+            int valid_last = pc.it.L - last_page * kPageRows;        // live rows of that page
+            asm volatile("" : "+r"(pj0), "+r"(pj1), "+r"(npages), "+r"(last_page), "+r"(valid_last));
             if (!(ok = __all_sync(0xffffffffu, wait(q_full, k & 1)))) break;
             if (!(ok = __all_sync(0xffffffffu, wait(k_full(gj % S::kStages), (gj / S::kStages) & 1)))) break;
-            for (int t = 0; ok && t < S::kQTiles; ++t) ok = issue_s(t, gj, it.ntiles == 1);
+            for (int t = 0; ok && t < S::kQTiles; ++t) ok = issue_s(t, gj, pj1 - pj0 == 1);
             // per KV tile j: O_A += P_A V(j), S_A(j + 1), O_B += P_B V(j), S_B(j + 1) -- the tensor
             // core works on one query tile while the other tile's softmax runs
-            for (int j = 0; ok && j < it.ntiles; ++j) {
-                const int gg = gj + j, s = gg % S::kStages;
+            for (int j = pj0; ok && j < pj1; ++j) {
+                const int gg = gj + (j - pj0), s = gg % S::kStages;
                 if (!(ok = __all_sync(0xffffffffu, wait(v_full(s), (gg / S::kStages) & 1)))) break;
                 // rows past the context in the sequence's last page may hold anything (NaN in free
                 // slots): zero their V before it meets a zero probability
-                if (last_page >= 8 * j && last_page < 8 * j + 8 && last_page < it.npages && valid_last < kPageRows) {
+                if (last_page >= 8 * j && last_page < 8 * j + 8 && last_page < npages && valid_last < kPageRows) {
                     const int pg = last_page - 8 * j;
                     const int nz = (kPageRows - valid_last) * 8;      // 16-byte pieces per chunk
                     for (int i = lane; i < 2 * nz; i += 32) {
@@ -354,17 +493,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     fence_proxy_async_shared();
                 }
                 __syncwarp();
-                const bool more = j + 1 < it.ntiles;
+                const bool more = j + 1 < pj1;
                 for (int t = 0; ok && t < S::kQTiles; ++t) {
                     // an item's first product overwrites O_t: the previous item's O_t has been read out
-                    if (j == 0 && k >= 1 && !(ok = __all_sync(0xffffffffu, wait(o_free(t), (k - 1) & 1)))) break;
-                    ok = issue_pv(t, gg, j == 0);
+                    if (j == pj0 && k >= 1 && !(ok = __all_sync(0xffffffffu, wait(o_free(t), (k - 1) & 1)))) break;
+                    ok = issue_pv(t, gg, j == pj0);
                     if (ok && more && t == 0)
                         ok = __all_sync(0xffffffffu, wait(k_full((gg + 1) % S::kStages), ((gg + 1) / S::kStages) & 1));
-                    if (ok && more) ok = issue_s(t, gg + 1, j + 2 == it.ntiles);
+                    if (ok && more) ok = issue_s(t, gg + 1, j + 2 == pj1);
                 }
             }
-            gj += it.ntiles;
+            gj += pj1 - pj0;
             ++k;
         }
         // every MMA issued has completed before TMEM is freed
@@ -382,15 +521,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const float sl = p.logit_scale_log2;
         int gj = 0;
         bool ok = true;
-        for (int ri = 0; ok; ++ri) {
-            const int item = item_index(ri);
-            if (item < 0) break;
-            PrefillItem it;
-            if (!item_info(item, it)) continue;
+        PrefillPiece pc;
+        while (ok && next_piece(pc)) {
+            const PrefillItem& it = pc.it;
             const bool valid = r < rows && qi < it.nq;
             const int prow = it.pos0 + min(qi, it.nq - 1);       // causal limit of the row
             float m_run = -INFINITY, l_run = 0.f;                // running maximum (exp2 domain) and sum
-            for (int j = 0; j < it.ntiles; ++j, ++gj) {
+            for (int j = pc.j0; j < pc.j1; ++j, ++gj) {
                 if (!(ok = __all_sync(0xffffffffu, wait(s_full(t), gj & 1)))) break;
                 tc_fence_after();
                 // pass 1: causal mask and maximum of the row's raw logits (four independent chains);
@@ -422,7 +559,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const float m_new = raise ? mt : m_run;
                 // O_t += P V of the previous KV tile completed before S_t of this one was issued, so
                 // O_t is final for it and may be rescaled; the item's first product overwrites O_t
-                if (j > 0 && __any_sync(0xffffffffu, raise)) {
+                if (j > pc.j0 && __any_sync(0xffffffffu, raise)) {
                     if (!(ok = __all_sync(0xffffffffu, wait(o_done(t), (gj - 1) & 1)))) break;
                     tc_fence_after();
                     const float alpha = raise ? fast_exp2(m_run - m_new) : 1.f;
@@ -472,24 +609,113 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_arrive(p_full(t));
             }
             if (!ok) break;
-            // ---- out = O_t / l ----
             if (!(ok = __all_sync(0xffffffffu, wait(o_done(t), (gj - 1) & 1)))) break;
             tc_fence_after();
-            const float inv = p.out_scale / l_run;
             __half* dst = p.out + ((int64_t)(it.qs0 + it.i0 + qi) * p.Hq + (int64_t)it.g * G + hh) * kHeadDim;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float o[32];
-                tmem_ld32(o_row + 32 * c, o);
-                if (valid) {
+            auto store_out = [&](int c, const float (&o)[32], float inv) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 u;
-                        u.x = pack_half2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-                        u.y = pack_half2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-                        u.z = pack_half2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-                        u.w = pack_half2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-                        *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q) = u;
+                for (int q = 0; q < 4; ++q) {
+                    uint4 u;
+                    u.x = pack_half2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+                    u.y = pack_half2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+                    u.z = pack_half2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+                    u.w = pack_half2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+                    *reinterpret_cast<uint4*>(dst + 32 * c + 8 * q) = u;
+                }
+            };
+            if (!kStream || (pc.j0 == 0 && pc.j1 == it.ntiles)) {
+                // ---- a whole item: out = O_t / l ----
+                const float inv = p.out_scale / l_run;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float o[32];
+                    tmem_ld32(o_row + 32 * c, o);
+                    if (valid) store_out(c, o, inv);
+                }
+                tc_fence_before();
+                mbar_arrive(o_free(t));                          // O_t may be overwritten
+                continue;
+            }
+            // ---- a piece of an item cut at a CTA boundary ----
+            // Every piece stores its (m, l, O) rows; a warp's ticket then counts its 32 rows, and the
+            // warp that takes the last ticket merges the pieces of those rows:
+            // M = max m_k, out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k. The merger's own O
+            // is still in TMEM (O_t is released after the ticket); the others' come from L2.
+            const int c_first = cta_of(pc.u), c_last = cta_of(pc.u + it.ntiles - 1);
+            // a piece's slot: 0 if it starts the range of CTA c, else 1 (the CTA's last piece)
+            auto part_of = [&](int c) -> uint8_t* {
+                const int slot = 2 * c + (max(pc.u, range_lo(c)) == range_lo(c) ? 0 : 1);
+                return ws + ((int64_t)slot * S::kQTiles + t) * S::kPartBytes;
+            };
+            auto ml_of = [&](int c) { return reinterpret_cast<const float2*>(part_of(c) + 128 * 128 * 4) + r; };
+            {
+                uint8_t* part = part_of((int)blockIdx.x);
+                float4* po = reinterpret_cast<float4*>(part);
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    float o[2][32];
+                    tmem_ld32x2(o_row + 64 * h, o[0], o_row + 64 * h + 32, o[1]);
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            __stcg(po + (16 * h + 8 * c2 + q) * 128 + r,
+                                   make_float4(o[c2][4 * q], o[c2][4 * q + 1], o[c2][4 * q + 2], o[c2][4 * q + 3]));
+                }
+                __stcg(reinterpret_cast<float2*>(part + 128 * 128 * 4) + r, make_float2(m_run, l_run));
+            }
+            // the warp barrier orders every lane's stores before lane 0's release-acquire ticket;
+            // the merger's loads follow its acquire
+            __syncwarp();
+            unsigned int* cnt = ws_count + ((int64_t)c_last * S::kQTiles + t) * 4 + quarter;
+            unsigned int prev = 0;
+            if (lane == 0) prev = atomic_add_acq_rel_gpu(cnt, 1u);
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            __syncwarp();
+            const int n_oth = c_last - c_first;                  // pieces besides this one
+            if (prev == (unsigned int)n_oth) {
+                if (lane == 0) *cnt = 0u;                        // ready for the next call
+                const int me = (int)blockIdx.x;
+                auto oth = [&](int k) { return c_first + k + (c_first + k >= me ? 1 : 0); };
+                float M = m_run;
+                if (valid)
+                    for (int k = 0; k < n_oth; ++k) M = fmaxf(M, __ldcg(ml_of(oth(k))).x);
+                const float w_self = fast_exp2(m_run - M);       // a piece that saw no position: 0
+                float den = l_run * w_self;
+                if (valid)
+                    for (int k = 0; k < n_oth; ++k) {
+                        const float2 a = __ldcg(ml_of(oth(k)));
+                        den += a.y * fast_exp2(a.x - M);
+                    }
+                const float inv = p.out_scale / den;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {                    // 64 channels at a time
+                    float o[2][32];
+                    tmem_ld32x2(o_row + 64 * h, o[0], o_row + 64 * h + 32, o[1]);
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[c2][i] *= w_self;
+                    if (valid) {
+#pragma unroll 1
+                        for (int k = 0; k < n_oth; ++k) {
+                            const uint8_t* part = part_of(oth(k));
+                            const float4* src = reinterpret_cast<const float4*>(part) + 16 * h * 128 + r;
+                            float4 v[16];
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) v[q] = __ldcg(src + q * 128);
+                            const float w = fast_exp2(__ldcg(reinterpret_cast<const float2*>(part + 128 * 128 * 4) + r).x - M);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                float* d = &o[q >> 3][4 * (q & 7)];
+                                d[0] = fmaf(w, v[q].x, d[0]);
+                                d[1] = fmaf(w, v[q].y, d[1]);
+                                d[2] = fmaf(w, v[q].z, d[2]);
+                                d[3] = fmaf(w, v[q].w, d[3]);
+                            }
+                        }
+                        store_out(2 * h, o[0], inv);
+                        store_out(2 * h + 1, o[1], inv);
                     }
                 }
             }

@@ -234,8 +234,16 @@ def test_prefill_rejects_bad_arguments_on_host(kw, status):
     a.update(kw)
     rc = pkv.load_library().paged_gqa_prefill_attention(
         a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["qs"], a["B"], a["total"], a["maxq"], a["Hq"],
-        a["Hkv"], a["D"], a["bs"], a["mb"], a["nb"], a["maxc"], a["scale"], a["dtype"], 1.0, 1.0, None)
+        a["Hkv"], a["D"], a["bs"], a["mb"], a["nb"], a["maxc"], a["scale"], a["dtype"], 1.0, 1.0, None, 0, None)
     assert rc == status
+
+
+@pytest.mark.parametrize("args", [(0, 2, 128, 0), (12, 0, 128, 0), (12, 5, 128, 0), (12, 2, 64, 0),
+                                  (36, 4, 128, 0), (12, 2, 128, 7), (12, 2, 128, 1)])
+def test_prefill_workspace_size_zero_without_a_schedule_to_serve(args):
+    """Invalid sizes and an FP8 cache (whose kernel takes no workspace) need none; the size of a valid
+    f16 call needs the device's SM count, so it is checked on the GPU."""
+    assert pkv.load_library().paged_gqa_prefill_workspace_size(*args) == 0
 
 
 def test_prefill_flops_closed_form():

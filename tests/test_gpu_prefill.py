@@ -30,17 +30,38 @@ def _case(name, seed, n_new, **sizes):
     return w, x, q, qs
 
 
-def _run(w, x, q, qs, kv_dtype="f16", kc=None, vc=None):
+# The two schedules of the f16 kernel: whole items (no workspace) and the load-balanced one that
+# cuts items at CTA boundaries and merges their pieces (a zero-filled workspace).
+SCHEDULES = ["items", "balanced"]
+PART_BYTES = 128 * 128 * 4 + 128 * 8           # one piece's partial rows of one query tile
+
+
+def _workspace(w):
+    n = pkv.paged_gqa_prefill_workspace_size(w.Hq, w.Hkv, w.head_dim)
+    assert n > 0
+    return torch.zeros(n, dtype=torch.uint8, device="cuda")
+
+
+def _run(w, x, q, qs, kv_dtype="f16", kc=None, vc=None, schedule="items", ws=None):
     out = torch.full(q.shape, float("nan"), dtype=torch.float16, device="cuda")
     kc = x["k_pool"] if kc is None else kc
     vc = x["v_pool"] if vc is None else vc
     n = qs[1:] - qs[:-1]
+    if schedule == "balanced" and ws is None:
+        ws = _workspace(w)
     pkv.paged_gqa_prefill_attention(out, dev(q), dev(kc), dev(vc), dev(x["block_tables"]), dev(x["context_lens"]),
                                     dev(qs), max_query_len=max(int(n.max()), 1),
                                     max_context_len=max(int(x["context_lens"].max()), 1),
                                     softmax_scale=float(x["softmax_scale"]), kv_dtype=kv_dtype,
-                                    k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]))
+                                    k_scale=float(x["k_scale"]), v_scale=float(x["v_scale"]),
+                                    workspace=ws if schedule == "balanced" else None)
     return host(out)
+
+
+def _tickets_clear(ws):
+    """The merge tickets (after the partial results of two slots x two tiles per SM) are back at 0."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return bool((ws[4 * sms * PART_BYTES:] == 0).all())
 
 
 def _oracle(w, x, q, qs, kv_dtype="f16", kc=None, vc=None):
@@ -56,9 +77,10 @@ def _oracle(w, x, q, qs, kv_dtype="f16", kc=None, vc=None):
     ("qwen2.5-7b", [9, 0, 64, 33], dict(B=4, num_blocks=2048)),                      # G = 7, a sequence without queries
     ("tiny", [17, 40], {}),
 ])
-def test_prefill_parity_f16(name, n_new, sizes):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_prefill_parity_f16(name, n_new, sizes, schedule):
     w, x, q, qs = _case(name, 3, n_new, **sizes)
-    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), f"{name} {n_new[:3]}")
+    assert_attention_close(_run(w, x, q, qs, schedule=schedule), _oracle(w, x, q, qs), f"{name} {n_new[:3]}")
     assert pkv.pkv_device_error() == 0
 
 
@@ -83,13 +105,15 @@ def test_one_query_per_sequence_matches_decode():
     assert_attention_close(host(out), ref, "decode")
 
 
-def test_long_chunked_prefill():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_long_chunked_prefill(schedule):
     """Two sequences append 256 tokens to contexts of up to 2048 (Qwen2.5-7B heads)."""
     w, x, q, qs = _case("qwen2.5-7b", 6, [256, 256], B=2, num_blocks=1024, ctx=("uniform", 1024, 2048))
-    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "long chunked prefill")
+    assert_attention_close(_run(w, x, q, qs, schedule=schedule), _oracle(w, x, q, qs), "long chunked prefill")
 
 
-def test_inconsistent_lengths_are_flagged_not_faulted():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_inconsistent_lengths_are_flagged_not_faulted(schedule):
     w, x, q, qs = _case("qwen2.5-1.5b", 8, [4, 4, 4], B=3, num_blocks=256, ctx=("fixed", (20, 3, 30)))
     # sequence 1 has a 3-token context; ask for 4 queries by moving the boundaries
     qs_bad = np.array([0, 4, 8, 12], np.int32)
@@ -97,7 +121,8 @@ def test_inconsistent_lengths_are_flagged_not_faulted():
     out = torch.full(q_bad.shape, 7.0, dtype=torch.float16, device="cuda")
     pkv.paged_gqa_prefill_attention(out, dev(q_bad), dev(x["k_pool"]), dev(x["v_pool"]), dev(x["block_tables"]),
                                     dev(x["context_lens"]), dev(qs_bad), max_query_len=4, max_context_len=30,
-                                    softmax_scale=float(x["softmax_scale"]))
+                                    softmax_scale=float(x["softmax_scale"]),
+                                    workspace=_workspace(w) if schedule == "balanced" else None)
     got = host(out)
     assert pkv.pkv_device_error() & pkv.DEVERR_CONTEXT_LEN
     assert (got[4:8] == 7.0).all()                  # the flagged sequence's rows are left alone
@@ -105,16 +130,18 @@ def test_inconsistent_lengths_are_flagged_not_faulted():
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (12, 4), (16, 4), (10, 2), (16, 2)])
-def test_prefill_group_sizes(Hq, Hkv):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_prefill_group_sizes(Hq, Hkv, schedule):
     """Every group size packs floor(128 / G) query tokens x G heads into the tile's rows
     (128, 64, 42, 32, 25 and 16 tokens); several tiles per sequence, a one-query sequence."""
     w, x, q, qs = _case("qwen2.5-1.5b", 9, [150, 1, 77], B=3, num_blocks=512, Hq=Hq, Hkv=Hkv,
                         ctx=("uniform", 150, 600))
-    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), f"Hq {Hq} / Hkv {Hkv}")
+    assert_attention_close(_run(w, x, q, qs, schedule=schedule), _oracle(w, x, q, qs), f"Hq {Hq} / Hkv {Hkv}")
     assert pkv.pkv_device_error() == 0
 
 
-def test_prefill_large_logits():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_prefill_large_logits(schedule):
     """Logits that grow along the sequence: q scaled by 3 and each key by 1 + position / 256, so
     the running maximum of a row rises by more than the rescale threshold (8 in the exp2 domain)
     several times over its KV tiles and the output accumulated so far is rescaled each time."""
@@ -126,21 +153,23 @@ def test_prefill_large_logits():
             pos = 16 * j + np.arange(16, dtype=np.float32)
             k[x["block_tables"][b, j]] *= (1 + pos / 256)[:, None, None]
     x["k_pool"] = k.astype(F16)                     # NaN rows stay NaN
-    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "large logits")
+    assert_attention_close(_run(w, x, q, qs, schedule=schedule), _oracle(w, x, q, qs), "large logits")
     assert pkv.pkv_device_error() == 0
 
 
-def test_prefill_zero_scale_is_the_causal_mean():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_prefill_zero_scale_is_the_causal_mean(schedule):
     """softmax_scale = 0: every query averages V over its causal window (masked entries stay out
     of the average even though 0 times their logit is 0)."""
     w, x, q, qs = _case("qwen2.5-7b", 11, [40, 150], B=2, num_blocks=512, ctx=("uniform", 200, 400))
     x["softmax_scale"] = np.float32(0.0)
-    assert_attention_close(_run(w, x, q, qs), _oracle(w, x, q, qs), "zero scale")
+    assert_attention_close(_run(w, x, q, qs, schedule=schedule), _oracle(w, x, q, qs), "zero scale")
     assert pkv.pkv_device_error() == 0
 
 
 @pytest.mark.parametrize("name", ["qwen2.5-7b", "qwen2.5-1.5b"])
-def test_prefill_more_items_than_ctas_sampled(name):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_prefill_more_items_than_ctas_sampled(name, schedule):
     """The bench's case at full size: 8 sequences append 512 tokens each to 2048-token contexts.
     At 7B heads that is 480 work items (two 18-token query tiles, KV head, sequence), at 1.5B heads
     208, more than the 148 CTAs of the persistent grid, so CTAs run several items each and carry
@@ -149,7 +178,7 @@ def test_prefill_more_items_than_ctas_sampled(name):
     length L_b - n_b + i + 1 over the same block table."""
     B, n_new, L = 8, 512, 2048
     w, x, q, qs = _case(name, 12, [n_new] * B, B=B, num_blocks=B * L // 16 + 64, ctx=("fixed", (L,) * B))
-    got = _run(w, x, q, qs)
+    got = _run(w, x, q, qs, schedule=schedule)
     rng = np.random.default_rng(13)
     rows = np.sort(np.concatenate([rng.choice(int(qs[-1]), 40, replace=False), [0, int(qs[-1]) - 1]]))
     b_of = np.searchsorted(qs, rows, side="right") - 1
@@ -159,3 +188,48 @@ def test_prefill_more_items_than_ctas_sampled(name):
     assert_attention_close(got[rows], ref, f"{name} sampled rows of {int(qs[-1])}")
     assert np.isfinite(got).all()
     assert pkv.pkv_device_error() == 0
+
+
+def test_balanced_items_cut_into_many_pieces():
+    """One long sequence: 300 queries at the end of a 6000-token context at 7B heads are 36 items of
+    about 47 KV tiles, so each CTA's share (about 11 tiles) cuts every item into 4 to 6 pieces: a
+    head piece (tile 0), middle pieces spanning a whole CTA, a tail piece. Rows whose position lies
+    before a tail piece's first tile see nothing there (maximum -inf, sum 0) and must get weight 0."""
+    w, x, q, qs = _case("qwen2.5-7b", 14, [300], B=1, num_blocks=512, ctx=("fixed", (6000,)))
+    ref = _oracle(w, x, q, qs)
+    ws = _workspace(w)
+    got = _run(w, x, q, qs, schedule="balanced", ws=ws)
+    assert_attention_close(got, ref, "many pieces")
+    assert pkv.pkv_device_error() == 0
+    assert _tickets_clear(ws)
+
+
+def test_balanced_workspace_is_reusable():
+    """Calls that complete leave the tickets at zero: the same workspace serves the next call, with
+    the same result bit for bit, and a different batch after it."""
+    w, x, q, qs = _case("qwen2.5-7b", 15, [100, 7, 260, 33], B=4, num_blocks=2048, ctx=("uniform", 300, 3000))
+    ws = _workspace(w)
+    first = _run(w, x, q, qs, schedule="balanced", ws=ws)
+    assert _tickets_clear(ws)
+    second = _run(w, x, q, qs, schedule="balanced", ws=ws)
+    assert np.array_equal(first.view(np.uint16), second.view(np.uint16))
+    assert_attention_close(second, _oracle(w, x, q, qs), "reused workspace")
+    w2, x2, q2, qs2 = _case("qwen2.5-7b", 16, [1, 64], B=2, num_blocks=512, ctx=("uniform", 64, 900))
+    assert_attention_close(_run(w2, x2, q2, qs2, schedule="balanced", ws=ws), _oracle(w2, x2, q2, qs2),
+                           "another batch on the same workspace")
+    assert pkv.pkv_device_error() == 0 and _tickets_clear(ws)
+
+
+def test_balanced_small_work_uses_fewer_ctas():
+    """Fewer KV tiles than 4 per SM: the schedule gives every CTA at least 4 and leaves the rest idle."""
+    w, x, q, qs = _case("qwen2.5-1.5b", 17, [5, 130, 1], B=3, num_blocks=256, ctx=("uniform", 130, 700))
+    assert_attention_close(_run(w, x, q, qs, schedule="balanced"), _oracle(w, x, q, qs), "few tiles")
+    assert pkv.pkv_device_error() == 0
+
+
+def test_balanced_workspace_too_small_is_rejected():
+    w, x, q, qs = _case("tiny", 18, [17, 40])
+    small = torch.zeros(pkv.paged_gqa_prefill_workspace_size(w.Hq, w.Hkv, w.head_dim) - 256, dtype=torch.uint8,
+                        device="cuda")
+    with pytest.raises(pkv.PagedKVError):
+        _run(w, x, q, qs, schedule="balanced", ws=small)
