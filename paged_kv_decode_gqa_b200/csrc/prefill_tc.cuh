@@ -234,9 +234,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int64_t per_g = seq_tiles(cb);
         cg = (int)((u_lo - s_first[1]) / per_g);
         cu = s_first[1] + cg * per_g;
-        PrefillItem it;
-        while (make_item(cb, cg, cq, it) > 0 && cu + it.ntiles <= u_lo) {
-            cu += it.ntiles;
+        // the query group holding u_lo: its sequence's lengths once, then arithmetic
+        const int L = __ldg(p.context_lens + cb);
+        const int n = __ldg(p.query_start + cb + 1) - __ldg(p.query_start + cb);
+        for (int i0 = 0; i0 < n; i0 += S::kQTiles * T) {
+            const int ntiles = (L - n + min(i0 + S::kQTiles * T, n) - 1) / S::kKvTok + 1;
+            if (cu + ntiles > u_lo) break;
+            cu += ntiles;
             ++cq;
         }
     }
@@ -677,25 +681,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (lane == 0) *cnt = 0u;                        // ready for the next call
                 const int me = (int)blockIdx.x;
                 auto oth = [&](int k) { return c_first + k + (c_first + k >= me ? 1 : 0); };
-                float M = m_run;
-                if (valid)
-                    for (int k = 0; k < n_oth; ++k) M = fmaxf(M, __ldcg(ml_of(oth(k))).x);
-                const float w_self = fast_exp2(m_run - M);       // a piece that saw no position: 0
-                float den = l_run * w_self;
-                if (valid)
-                    for (int k = 0; k < n_oth; ++k) {
-                        const float2 a = __ldcg(ml_of(oth(k)));
-                        den += a.y * fast_exp2(a.x - M);
-                    }
-                const float inv = p.out_scale / den;
+                // online log-sum-exp over the pieces, 64 channels at a time: each other piece's
+                // (m, l) comes with its 64 values in one round trip
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {                    // 64 channels at a time
+                for (int h = 0; h < 2; ++h) {
                     float o[2][32];
                     tmem_ld32x2(o_row + 64 * h, o[0], o_row + 64 * h + 32, o[1]);
-#pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[c2][i] *= w_self;
+                    float M = m_run, den = l_run;
                     if (valid) {
 #pragma unroll 1
                         for (int k = 0; k < n_oth; ++k) {
@@ -704,16 +696,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             float4 v[16];
 #pragma unroll
                             for (int q = 0; q < 16; ++q) v[q] = __ldcg(src + q * 128);
-                            const float w = fast_exp2(__ldcg(reinterpret_cast<const float2*>(part + 128 * 128 * 4) + r).x - M);
+                            const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + 128 * 128 * 4) + r);
+                            // a piece that saw no position has m = -inf, l = 0 and O = 0
+                            const float m_new = fmaxf(M, ml.x);
+                            const float a = M == m_new ? 1.f : fast_exp2(M - m_new);
+                            const float w = ml.x == m_new ? 1.f : fast_exp2(ml.x - m_new);
+                            den = fmaf(den, a, w * ml.y);
 #pragma unroll
                             for (int q = 0; q < 16; ++q) {
                                 float* d = &o[q >> 3][4 * (q & 7)];
-                                d[0] = fmaf(w, v[q].x, d[0]);
-                                d[1] = fmaf(w, v[q].y, d[1]);
-                                d[2] = fmaf(w, v[q].z, d[2]);
-                                d[3] = fmaf(w, v[q].w, d[3]);
+                                d[0] = fmaf(d[0], a, w * v[q].x);
+                                d[1] = fmaf(d[1], a, w * v[q].y);
+                                d[2] = fmaf(d[2], a, w * v[q].z);
+                                d[3] = fmaf(d[3], a, w * v[q].w);
                             }
+                            M = m_new;
                         }
+                        const float inv = p.out_scale / den;
                         store_out(2 * h, o[0], inv);
                         store_out(2 * h + 1, o[1], inv);
                     }
