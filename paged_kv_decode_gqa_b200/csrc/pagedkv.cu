@@ -714,9 +714,6 @@ bool make_q_map(CUtensorMap* map, const void* q, int Hq, int total, int G, int t
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// f16 prefill on tcgen05: a persistent grid of one CTA per SM (its shared
-// memory and TMEM) over items of (two tiles of 128 / G query tokens, KV head,
-// sequence).
 // Workspace of the stream-K prefill schedule for a device of `ctas` SMs (grids of up to one CTA
 // per SM): two partial results (both query tiles) per CTA, then one ticket per (CTA, query tile,
 // row quarter).
@@ -732,6 +729,10 @@ PrefillWorkspace prefill_layout(int64_t ctas) {
     return w;
 }
 
+// f16 prefill on tcgen05: a persistent grid of one CTA per SM (its shared
+// memory and TMEM) over items of (two tiles of 128 / G query tokens, KV head,
+// sequence); whole items without a workspace, the load-balanced (stream-K)
+// schedule with one.
 pkv_status launch_prefill_tc(const pkv::PrefillParams& prm, const CUtensorMap& mk, const CUtensorMap& mv,
                              int max_query_len, int Hkv, int B, void* workspace, size_t workspace_bytes,
                              cudaStream_t stream) {
