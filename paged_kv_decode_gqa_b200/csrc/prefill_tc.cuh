@@ -365,8 +365,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (warp == S::kTmaKWarp || warp == S::kTmaVWarp) {
         // ============================ TMA: K or V ============================
-        // KV tiles are numbered across the CTA's items (gj); the K warp also loads each item's Q
-        // once the previous item's last S has read the buffers.
+        // KV tiles are numbered across the CTA's pieces (gj); the K warp also loads each piece's Q
+        // once the previous piece's last S has read the buffers.
         const bool is_k = warp == S::kTmaKWarp;
         if (lane == 0) {
             prefetch_tensormap(is_k ? &tm_k : &tm_v);
@@ -426,7 +426,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         constexpr uint32_t kIdescS = umma_idesc_f16(128, 128, 0);    // Q K^T: both K-major
         constexpr uint32_t kIdescPV = umma_idesc_f16(128, 128, 1);   // P V: V is MN-major
         // S_t = Q_t K^T of global KV tile gg, once O_t += P_t V of tile gg - 1 has read P_t out
-        // of S_t; `last`: the item's last tile, after which Q may be reloaded
+        // of S_t; `last`: the piece's last tile, after which Q may be reloaded
         auto issue_s = [&](int t, int gg, bool last) -> bool {
             if (gg >= 1 && !__all_sync(0xffffffffu, wait(o_done(t), (gg - 1) & 1))) return false;
             tc_fence_after();
@@ -447,7 +447,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             return true;
         };
-        // O_t += P_t V of global KV tile gg, P_t read from TMEM; `first`: the item's first tile,
+        // O_t += P_t V of global KV tile gg, P_t read from TMEM; `first`: the piece's first tile,
         // whose product overwrites O_t
         auto issue_pv = [&](int t, int gg, bool first) -> bool {
             const int s = gg % S::kStages;
@@ -499,7 +499,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 __syncwarp();
                 const bool more = j + 1 < pj1;
                 for (int t = 0; ok && t < S::kQTiles; ++t) {
-                    // an item's first product overwrites O_t: the previous item's O_t has been read out
+                    // a piece's first product overwrites O_t: the previous piece's O_t has been read out
                     if (j == pj0 && k >= 1 && !(ok = __all_sync(0xffffffffu, wait(o_free(t), (k - 1) & 1)))) break;
                     ok = issue_pv(t, gg, j == pj0);
                     if (ok && more && t == 0)
@@ -562,7 +562,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const bool raise = mt > m_run + S::kRescaleThreshold;
                 const float m_new = raise ? mt : m_run;
                 // O_t += P V of the previous KV tile completed before S_t of this one was issued, so
-                // O_t is final for it and may be rescaled; the item's first product overwrites O_t
+                // O_t is final for it and may be rescaled; the piece's first product overwrites O_t
                 if (j > pc.j0 && __any_sync(0xffffffffu, raise)) {
                     if (!(ok = __all_sync(0xffffffffu, wait(o_done(t), (gj - 1) & 1)))) break;
                     tc_fence_after();
