@@ -15,7 +15,8 @@
  * projection that produce the step's q and new K/V; paged_kv_fp8_scales and
  * the *_fp8_scaled variants, FP8 caches with scales on the device; and
  * paged_gqa_prefill_attention, many query tokens per sequence over the same
- * paged cache (chunked prefill).
+ * paged cache (chunked prefill), load-balanced over the SMs when given the
+ * workspace paged_gqa_prefill_workspace_size names.
  *
  * Sources, cited by page title and section:
  *  - "rvLLM 소개" (discuss.pytorch.kr), §PagedAttention과 FlashAttention-3:
