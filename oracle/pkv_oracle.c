@@ -386,13 +386,27 @@ int oracle_paged_prefill(double* out, double* lse, const uint16_t* q, const void
     float* vs = (float*)malloc(sizeof(float) * (size_t)Hkv);
     for (int g = 0; g < Hkv; ++g) { ks[g] = k_scale; vs[g] = v_scale; }
     int status = 0;
-#pragma omp parallel for schedule(dynamic)
-    for (int b = 0; b < B; ++b) {
-        int n = query_start[b + 1] - query_start[b], L = context_lens[b];
-        const int32_t* bt_row = block_tables + (int64_t)b * max_blocks_per_seq;
-        double* s = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
-        for (int i = 0; i < n; ++i) {
-            int64_t row = query_start[b] + i;
+    int max_L = 1;
+    for (int b = 0; b < B; ++b) max_L = context_lens[b] > max_L ? context_lens[b] : max_L;
+    const int64_t total = B > 0 ? query_start[B] : 0;
+    /* query rows are independent: one row per iteration, any thread (the arithmetic of a row does
+     * not depend on which thread computes it) */
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)max_L);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t row = 0; row < total; ++row) {
+            /* the row's sequence: the last b with query_start[b] <= row (sequences without
+             * queries share their start with the next one) */
+            int lo = 0, hi = B;                     /* query_start[lo] <= row < query_start[hi] */
+            while (hi - lo > 1) {
+                int mid = (lo + hi) / 2;
+                if (query_start[mid] <= row) lo = mid; else hi = mid;
+            }
+            const int b = lo;
+            const int n = query_start[b + 1] - query_start[b], L = context_lens[b];
+            const int32_t* bt_row = block_tables + (int64_t)b * max_blocks_per_seq;
+            const int i = (int)(row - query_start[b]);
             int pos = L - n + i;                    /* R12: this query's position */
             const uint16_t* q_row = q + row * Hq * D;
             for (int h = 0; h < Hq; ++h) {
