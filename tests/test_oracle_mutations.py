@@ -56,7 +56,8 @@ MUTATIONS = {
     # paged prefill
     "prefill_causal_off_by_one": ("0, pos + 1)) {", "0, pos + (pos == 0))) {"),
     "prefill_position_from_start": ("int pos = L - n + i;", "int pos = i;"),
-    "prefill_rows_reversed": ("int64_t row = query_start[b] + i;", "int64_t row = query_start[b + 1] - 1 - i;"),
+    "prefill_rows_reversed": ("const int i = (int)(row - query_start[b]);",
+                              "const int i = (int)(query_start[b + 1] - 1 - row);"),
 }
 
 PIN_TESTS = [
